@@ -1,0 +1,484 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 GSA layer (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
+                    [--config pi3_f1000] [--dense full|off] [--no-e2e]
+
+A step is one full GSA forward (pool, compressed attention + streaming top-k,
+selection, upsample/gate/blend, special tokens) over the
+1000-frame pi^3-style workload (1000 frames x 36x36 patches + 5 special tokens
+per frame, 16 heads, d=64, s=4, top-32), inputs resident in HBM.  Inputs are
+7.9 GB per GPU, far above the 126 MB L2, so no flush is needed between steps.
+Under torchrun every rank runs its own independent copy of the workload (the
+layer has no cross-GPU exchange; heads and layers are independent), so per-GPU
+work is fixed as N grows ("weak" scaling) and `value` sums all ranks.
+
+--impl reference times the CPU oracle (fp64 numpy, as it stands) on a bounded
+sample of the same workload and reports the same metric; the other ranks of a
+multi-rank launch exit without work.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+from datetime import timedelta
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "GSA layer image tokens/s at 1000 views; % of bf16 peak; speedup vs dense attn"
+UNIT = "image tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# kernels of one step (names reported by gsa_get_kernel_times) and how each is graded
+TENSOR_KERNELS = {"comp_attn_topk", "special", "dense"}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_desc(cfg):
+    return (f"{cfg.name}: {cfg.num_frames} frames x {cfg.grid_h}x{cfg.grid_w} patch grid"
+            + (f" (padded {cfg.pad_h}x{cfg.pad_w})" if (cfg.pad_h, cfg.pad_w) != (cfg.grid_h, cfg.grid_w) else "")
+            + f" + {cfg.num_special} special tokens/frame, {cfg.num_heads} heads, d={cfg.head_dim},"
+            f" s={cfg.pool_s}, top-{cfg.topk}" + (f", fixed frames {list(cfg.fixed_frames)}" if cfg.fixed_frames else ""))
+
+
+def algorithmic_work(cfg, kc):
+    """Per-launch algorithmic FLOPs and compulsory HBM bytes of each kernel."""
+    H, d = cfg.num_heads, cfg.head_dim
+    R = cfg.num_regions
+    M = cfg.num_img_valid
+    slots = cfg.num_img_slots
+    Ms = cfg.num_spec
+    e = 2 if cfg.dtype == "bf16" else 4
+    s2 = cfg.pool_s ** 2
+    nfix_keys = len(cfg.fixed_frames) * (cfg.num_special + cfg.grid_h * cfg.grid_w)
+    keys_sel = cfg.topk * s2 + nfix_keys
+    w = {}
+    # pool reads Q/K/V once and writes bf16 Q/K/V_comp plus the bf16 low parts of Q/K_comp
+    w["pool"] = {"flops": 0.0,
+                 "bytes": 3.0 * H * slots * d * e + 5.0 * H * R * d * e}
+    # the guide scores take three bf16 products (hi*hi + hi*lo + lo*hi); the
+    # algorithmic count is the plain 4*d per (query, key) pair of one attention
+    w["comp_attn_topk"] = {"flops": 4.0 * d * R * R * H,
+                           "bytes": 5.0 * H * R * d * e + H * R * d * 4 + H * R * kc * 4}
+    w["selection"] = {"flops": 4.0 * d * M * keys_sel * H,
+                      # Q_img + O_sel + every image token's K/V once + idx
+                      "bytes": 2.0 * H * slots * d * e + 2.0 * H * slots * d * e + H * R * cfg.topk * 4}
+    w["epilogue"] = {"flops": 2.0 * d * d * M * H,
+                     "bytes": 3.0 * H * slots * d * e + H * R * d * 4 + H * d * d * e}
+    w["special"] = {"flops": 4.0 * d * Ms * (Ms + M) * H, "bytes": 2.0 * H * (Ms + slots) * d * e + 2.0 * H * Ms * d * e}
+    w["special_merge"] = {"flops": 0.0, "bytes": 0.0}
+    w["dense"] = {"flops": 4.0 * d * (M + Ms) ** 2 * H, "bytes": 4.0 * H * (slots + Ms) * d * e}
+    return w
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sparse_global_attention_b200", "csrc")
+    for n in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, n), "rb") as f:
+            h.update(n.encode())
+            h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+def read_traffic(kernel, workload):
+    """dram bytes per launch recorded from an ncu capture of the current kernel
+    sources (profiles/ncu_traffic.txt: `kernel workload bytes source_sha`)."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    sha = kernel_source_sha()
+    with open(p) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) == 4 and not line.startswith("#") and parts[0] == kernel and parts[1] == workload:
+                return float(parts[2]) if parts[3] == sha else None
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            p = [x.strip() for x in ln.split(",")]
+            if len(p) < 7:
+                continue
+            try:
+                sm.append(float(p[0]))
+                mx = max(mx, float(p[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, p[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------
+# the CPU oracle as the baseline / reference arm
+# ---------------------------------------------------------------------------------------
+def oracle_sample(cfg, head_arrays, nwin, seed=0):
+    """Time the oracle on head 0: the head's full pooling plus `nwin` windows
+    (compressed row, top-k, selection, gate) and a proportional number of
+    special rows; extrapolate to the whole layer (every window of every head)."""
+    import numpy as np
+    import oracle
+    a = head_arrays
+    rng = np.random.default_rng(seed)
+    R = cfg.num_regions
+    win = np.sort(rng.choice(R, size=min(nwin, R), replace=False))
+    nspec = max(1, int(round(cfg.num_spec * len(win) / R))) if cfg.num_special else 0
+    srows = np.sort(rng.choice(cfg.num_spec, size=nspec, replace=False)) if nspec else np.zeros(0, int)
+    t0 = time.perf_counter()
+    for t in ("q_img", "k_img", "v_img"):
+        oracle.pool(a[t], cfg.grid_h, cfg.grid_w, cfg.pool_s)
+    t_pool = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.gsa_head(a["q_spec"], a["k_spec"], a["v_spec"], a["q_img"], a["k_img"], a["v_img"], a["w_g"],
+                    grid_h=cfg.grid_h, grid_w=cfg.grid_w, pool_s=cfg.pool_s, topk=cfg.topk,
+                    fixed_frames=cfg.fixed_frames, windows=win, spec_rows=srows)
+    t_all = time.perf_counter() - t0
+    t_win = max(t_all - t_pool, 1e-9)
+    per_head = t_pool + t_win * (R / len(win))
+    layer_s = per_head * cfg.num_heads
+    return {"layer_s": layer_s, "sample_s": t_pool + t_all, "windows": len(win), "spec_rows": nspec}
+
+
+def cpu_info():
+    cores = len(os.sched_getaffinity(0))
+    threads = None
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        blas = [f"{i.get('internal_api')}:{i.get('num_threads')}" for i in info if i.get("user_api") == "blas"]
+        threads = max([i.get("num_threads", 0) for i in info if i.get("user_api") == "blas"] or [cores])
+        return cores, threads, ",".join(blas)
+    except Exception:
+        return cores, cores, "unknown"
+
+
+def host_head_arrays(cfg, x, h=0):
+    from gsa_inputs import to_f64_numpy
+    return {k: to_f64_numpy(v[h]) for k, v in x.items()}
+
+
+def run_reference(args, cfg, rank, world):
+    """--impl reference: the CPU oracle as it stands, bounded samples of the workload."""
+    if rank != 0:
+        return None
+    from gsa_inputs import make_inputs
+    x = make_inputs(cfg, seed=0, device="cpu", heads=[0])
+    a = host_head_arrays(cfg, x, 0)
+    del x
+    nwin = args.ref_windows
+    for _ in range(args.warmup):
+        oracle_sample(cfg, a, nwin)
+    times, samples = [], []
+    for i in range(args.steps):
+        r = oracle_sample(cfg, a, nwin, seed=i)
+        times.append(r["layer_s"])
+        samples.append(r["sample_s"])
+    layer_s = statistics.median(times)
+    value = cfg.num_img_valid / layer_s
+    cores, threads, blas = cpu_info()
+    sample = (f"head 0 of {cfg.num_heads}: full pooling of the head + {nwin} random windows (compressed row,"
+              f" top-k, selection, gate) + proportional special rows; time extrapolated x{cfg.num_regions}/{nwin}"
+              f" windows and x{cfg.num_heads} heads; median of {args.steps} samples ({statistics.median(samples):.1f}"
+              f" s each); BLAS {blas}")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": layer_s * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": workload_desc(cfg), "parallelism": "cpu oracle, rank 0"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    return line
+
+
+# ---------------------------------------------------------------------------------------
+# the B200 arm
+# ---------------------------------------------------------------------------------------
+def run_b200(args, cfg, rank, world, local, dist):
+    import torch
+    import sparse_global_attention_b200 as gsa
+    from gsa_inputs import make_inputs
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    x = make_inputs(cfg, seed=rank, device=dev)
+    layer = gsa.GSALayer.from_workload(cfg)
+    out = {"o_img": torch.empty_like(x["q_img"]), "o_spec": torch.empty_like(x["q_spec"])}
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        layer.forward(x, out=out)
+    torch.cuda.synchronize()
+    st = layer.status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} during warm-up: {gsa.gsa_strerror(st)}")
+
+    # ---- timed region: K steps, inputs resident in HBM ------------------------
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            layer.forward(x, out=out)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    value = world * cfg.num_img_valid / (ms / 1e3)
+
+    # ---- per-kernel times (CUDA events recorded by the library on its stream) --
+    gsa.gsa_set_profiling(layer.ctx, True)
+    per = {}
+    nprof = max(1, min(args.steps, 5))
+    for _ in range(nprof):
+        layer.forward(x, out=out)
+        for name, t in gsa.gsa_get_kernel_times(layer.ctx):
+            per.setdefault(name, []).append(t)
+    gsa.gsa_set_profiling(layer.ctx, False)
+    kernel_ms = {k: statistics.mean(v) for k, v in per.items()}
+    launches_per_step = len(kernel_ms)
+    kc = cfg.topk
+
+    pk, pk_kind = peaks()
+    work = algorithmic_work(cfg, kc)
+    kernels = {}
+    for k, t in kernel_ms.items():
+        w = work.get(k, {"flops": 0.0, "bytes": 0.0})
+        ent = {"ms": round(t, 4)}
+        if w["flops"]:
+            ent["tflops"] = round(w["flops"] / (t / 1e3) / 1e12, 2)
+        if w["bytes"]:
+            ent["gbs"] = round(w["bytes"] / (t / 1e3) / 1e9, 1)
+        kernels[k] = ent
+    dom = max(kernel_ms, key=kernel_ms.get)
+    tpeak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+    if dom in TENSOR_KERNELS:
+        ach = work[dom]["flops"] / (kernel_ms[dom] / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(ach, 2), "peak": tpeak, "unit": "TFLOP/s"}
+    else:
+        ach = work[dom]["bytes"] / (kernel_ms[dom] / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s"}
+    roof["frac"] = round(ach / roof["peak"], 4)
+    roof["kernel"] = dom
+    roof["peak_source"] = f"{pk_kind} ({'sustained' if roof['bound'] == 'tensor' else 'copy'})"
+    roof["traffic"] = read_traffic(dom, cfg.name)
+    tensor_flops = sum(work[k]["flops"] for k in ("comp_attn_topk", "special", "selection", "epilogue"))
+    pct_peak = tensor_flops / (ms / 1e3) / 1e12 / tpeak
+
+    # ---- dense global attention of the same shape (speedup denominator) ---------
+    dense = None
+    if args.dense != "off" and rank == 0:
+        H, F, d = cfg.num_heads, cfg.num_frames, cfg.head_dim
+
+        def dense_layout(spec, img):
+            return torch.cat([spec, img.reshape(H, F, -1, d)], dim=2).reshape(H, -1, d).contiguous()
+
+        del out
+        torch.cuda.empty_cache()
+        qd, kd, vd = (dense_layout(x[n + "_spec"], x[n + "_img"]) for n in "qkv")
+        od = torch.empty_like(qd)
+        small = gsa.GSALayer.from_workload(cfg.with_(num_frames=2))
+        small.dense(qd[:, :2 * (cfg.num_special + cfg.pad_h * cfg.pad_w)].contiguous(),
+                    kd[:, :2 * (cfg.num_special + cfg.pad_h * cfg.pad_w)].contiguous(),
+                    vd[:, :2 * (cfg.num_special + cfg.pad_h * cfg.pad_w)].contiguous())
+        torch.cuda.synchronize()
+        small.close()
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        layer.dense(qd, kd, vd, od)
+        d1.record(stream)
+        torch.cuda.synchronize()
+        dms = d0.elapsed_time(d1)
+        dfl = work["dense"]["flops"]
+        dense = {"ms": round(dms, 2), "tflops": round(dfl / (dms / 1e3) / 1e12, 1),
+                 "frac": round(dfl / (dms / 1e3) / 1e12 / tpeak, 4), "reps": 1}
+        del qd, kd, vd, od
+        torch.cuda.empty_cache()
+        out = {"o_img": torch.empty_like(x["q_img"]), "o_spec": torch.empty_like(x["q_spec"])}
+    else:
+        pass
+    if dist is not None:
+        barrier()
+
+    # ---- end to end through the public API with host buffers ---------------------
+    e2e = None
+    if not args.no_e2e:
+        if "out" not in locals() or out is None:
+            out = {"o_img": torch.empty_like(x["q_img"]), "o_spec": torch.empty_like(x["q_spec"])}
+        hx = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in x.items()}
+        for k in hx:
+            hx[k].copy_(x[k])
+        ho = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in out.items()}
+        h2d = sum(t.numel() * t.element_size() for t in hx.values())
+        d2h = sum(t.numel() * t.element_size() for t in ho.values())
+
+        def e2e_step():
+            for k in hx:
+                x[k].copy_(hx[k], non_blocking=True)
+            layer.forward(x, out=out)
+            for k in ho:
+                ho[k].copy_(out[k], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ke = max(1, min(args.steps, 5))
+        f0.record(stream)
+        for _ in range(ke):
+            e2e_step()
+        f1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ems = max_over_ranks(f0.elapsed_time(f1) / ke)
+        e2e = {"value": world * cfg.num_img_valid / (ems / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": round(ems, 3), "steps": ke}
+
+    st = layer.status()
+    if st != 0:
+        raise RuntimeError(f"device status {st}: {gsa.gsa_strerror(st)}")
+
+    # ---- the oracle on the host cores (rank 0, N = 1 only) --------------------------
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        a = host_head_arrays(cfg, x, 0)
+        r = oracle_sample(cfg, a, args.cpu_windows)
+        cores, threads, blas = cpu_info()
+        cpu = {"value": cfg.num_img_valid / r["layer_s"], "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": (f"head 0 of {cfg.num_heads} of the same inputs: full pooling of the head + "
+                          f"{r['windows']} random windows (compressed row, top-k, selection, gate) + "
+                          f"{r['spec_rows']} special rows, {r['sample_s']:.1f} s of CPU work, extrapolated to "
+                          f"all windows and heads; BLAS {blas}; {cores} cores visible")}
+
+    layer.close()
+    if rank != 0:
+        return None
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+        "config": {"workload": workload_desc(cfg), "image_tokens": cfg.num_img_valid,
+                   "special_tokens": cfg.num_spec, "regions": cfg.num_regions,
+                   "l2": "inputs 7.9 GB per GPU >> 126 MB L2: no flush between steps",
+                   "parallelism": f"{world} independent replica(s), one per GPU, no collective on the data path"},
+        "roofline": roof, "pct_bf16_peak": round(pct_peak, 4),
+        "speedup_vs_dense": (round(dense["ms"] / ms, 2) if dense else None), "dense": dense,
+        "kernels": kernels, "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(), "e2e": e2e, "cpu_baseline": cpu,
+    }
+    return line
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--config", default="pi3_f1000")
+    ap.add_argument("--dense", default="full", choices=["full", "off"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-windows", type=int, default=2048)
+    ap.add_argument("--ref-windows", type=int, default=512)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "b200":
+        args.warmup = 3
+
+    from gsa_inputs import CONFIGS
+    cfg = CONFIGS[args.config]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if args.impl == "reference":
+        line = run_reference(args, cfg, rank, world)
+    else:
+        if world > 1:
+            import torch
+            import torch.distributed as dist_mod
+            torch.cuda.set_device(local)
+            dist_mod.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                        device_id=torch.device("cuda", local))
+            dist = dist_mod
+        line = run_b200(args, cfg, rank, world, local, dist)
+        if dist is not None:
+            dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

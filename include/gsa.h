@@ -1,0 +1,160 @@
+/*
+ * gsa.h -- C ABI of the B200 (sm_100a) Global Sparse Attention (GSA) layer.
+ *
+ * The layer is the one described in "Speed3R: Sparse Feed-forward 3D
+ * Reconstruction Models" (Paper-Notes, CVPR 2026), section "全局稀疏注意力
+ * （GSA）核心设计" (GSA core design):
+ *   - Q/K/V are split into special tokens and image tokens (equation for
+ *     Q = [Q_spec; Q_img]);
+ *   - special tokens attend densely to every token (equation for O_spec);
+ *   - image tokens take two branches: a compression branch (s x s mean
+ *     pooling, attention among the pooled tokens, guide scores
+ *     S_guide = Q_comp K_comp^T, nearest upsampling) and a selection branch
+ *     (top-k regions per compressed query, attention of the window's queries
+ *     to the full-resolution tokens of those regions);
+ *   - a gate g = sigmoid(W_g Q_img) mixes them: O_img = g*O_comp + (1-g)*O_sel.
+ * The VGGT variant (section "Speed3R-VGGT 适配") adds a fixed global context
+ * to the selection branch: every token of the reference frame and of frames
+ * sampled every 100 frames.
+ *
+ * Everything here is plain C: pointers and sizes, no framework types.
+ * Device pointers are CUDA device addresses owned by the caller; the context
+ * owns its workspace (device memory allocated in gsa_create).
+ * Streams are passed as void* holding a cudaStream_t (NULL = legacy default).
+ * Every call returns an int status (GSA_OK = 0); nothing aborts the process
+ * and no C++ exception crosses this boundary.
+ */
+#ifndef GSA_B200_H
+#define GSA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GSA_API __attribute__((visibility("default")))
+#else
+#define GSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* status codes */
+#define GSA_OK                 0
+#define GSA_ERR_INVALID_ARG    1  /* NULL pointer, negative size, bad enum          */
+#define GSA_ERR_SHAPE          2  /* grid not divisible by pool_s, head_dim != 64,
+                                     topk outside [1, candidates], region with no
+                                     valid token                                      */
+#define GSA_ERR_UNSUPPORTED    3  /* valid but not implemented (e.g. topk > 64)       */
+#define GSA_ERR_OOM            4  /* workspace allocation failed                      */
+#define GSA_ERR_CUDA           5  /* a CUDA runtime call failed                       */
+#define GSA_ERR_DEVICE_TIMEOUT 6  /* a bounded device-side wait ran out               */
+#define GSA_ERR_DEVICE_BOUNDS  7  /* a device-side index check failed                 */
+
+/* element type of every input and output of one context */
+#define GSA_BF16 0
+#define GSA_FP32 1
+
+/* gate modes: LEARNED uses g = sigmoid(W_g q); the other two force g = 1
+ * (compression branch only) or g = 0 (selection branch only).  They isolate
+ * the branches for testing (section "门控聚合", gated aggregation).         */
+#define GSA_GATE_LEARNED   0
+#define GSA_GATE_COMP_ONLY 1
+#define GSA_GATE_SEL_ONLY  2
+
+/* maximum top-k and maximum number of fixed-context frames */
+#define GSA_MAX_TOPK         64
+#define GSA_MAX_FIXED_FRAMES 16
+
+typedef struct gsa_ctx gsa_ctx;
+
+typedef struct {
+    int num_frames;        /* F >= 1                                              */
+    int grid_h, grid_w;    /* valid patch grid per frame                          */
+    int pad_h, pad_w;      /* stored grid, >= grid, divisible by pool_s; pad
+                              tokens sit at the bottom rows / right cols          */
+    int num_special;       /* special tokens per frame, >= 0 (0 = registers and
+                              camera tokens removed, pi^3 adaptation)             */
+    int num_heads;         /* H >= 1                                              */
+    int head_dim;          /* must be 64                                          */
+    int pool_s;            /* s in {1, 2, 4, 8} (bf16 path: {2, 4})               */
+    int topk;              /* regions per compressed query, 1..min(64, candidates) */
+    int dtype;             /* GSA_BF16 or GSA_FP32                                */
+    const int *fixed_frames; /* VGGT fixed global context frames (copied at
+                              create); NULL with num_fixed_frames = 0 for pi^3   */
+    int num_fixed_frames;
+    int gate_mode;         /* GSA_GATE_*                                          */
+    float softmax_scale;   /* 0 => 1/sqrt(head_dim)                               */
+} gsa_config;
+
+/* Validate `cfg` and create a context on the current CUDA device; allocates
+ * the workspace (gsa_workspace_bytes).  On error *out is set to NULL. */
+GSA_API int gsa_create(const gsa_config *cfg, gsa_ctx **out);
+
+/* Bytes of device workspace a context with this config allocates (0 if the
+ * config is invalid). */
+GSA_API size_t gsa_workspace_bytes(const gsa_config *cfg);
+
+/* One forward pass of the GSA layer, enqueued on `stream` (asynchronous: no
+ * host synchronisation, no allocation).
+ *   q_spec, k_spec, v_spec : [H][F][num_special][64]   (ignored if num_special=0)
+ *   q_img,  k_img,  v_img  : [H][F][pad_h][pad_w][64]
+ *   w_g                    : [H][64][64], row = output channel, no bias
+ *   o_spec                 : [H][F][num_special][64]   output
+ *   o_img                  : [H][F][pad_h][pad_w][64]  output; pad tokens get 0
+ *   sel_idx_out            : optional [H][R][topk] int32 output, R =
+ *                            F*(pad_h/s)*(pad_w/s); per row the selected regions
+ *                            ordered by guide score descending, then index
+ *                            ascending; NULL = not written
+ * All tensors are contiguous, in the context's dtype, on the context's device.
+ * One context serves one stream at a time.  Returns GSA_ERR_CUDA if a launch
+ * fails; device-side errors surface at gsa_get_status. */
+GSA_API int gsa_forward(gsa_ctx *ctx,
+                const void *q_spec, const void *k_spec, const void *v_spec,
+                const void *q_img, const void *k_img, const void *v_img,
+                const void *w_g, void *o_spec, void *o_img, int32_t *sel_idx_out,
+                void *stream);
+
+/* Dense global attention over every token of the same shape (the comparison
+ * baseline, "Full Attn." in the notes' latency table):
+ *   q, k, v, o : [H][F*(num_special + pad_h*pad_w)][64], per frame the special
+ *                tokens then the padded image grid.  Pad tokens are never used
+ *                as keys and their output rows are 0. */
+GSA_API int gsa_dense_forward(gsa_ctx *ctx, const void *q, const void *k, const void *v,
+                      void *o, void *stream);
+
+/* Device pointer and size of an intermediate of the last gsa_forward, for
+ * tests and profiling (valid until the next forward or gsa_destroy).
+ * which: 0 Q_comp, 1 K_comp, 2 V_comp  (context dtype, [H][R][64])
+ *        3 O'_comp (fp32, [H][R][64])
+ *        4 selected regions (int32, [H][R][topk])
+ *        5 O_sel (context dtype, [H][F][pad_h][pad_w][64])
+ *        6, 7 low parts of Q_comp, K_comp: bf16 contexts keep the pooled
+ *          value x as bf16 hi = bf16(x) (items 0, 1) plus lo = bf16(x - hi)
+ *          ([H][R][64] bf16), fp32 contexts return items 0, 1 again */
+GSA_API int gsa_get_intermediate(gsa_ctx *ctx, int which, void **dev_ptr, size_t *bytes);
+
+/* Per-kernel timing: when enabled, gsa_forward records CUDA events on its
+ * stream around each kernel; gsa_get_kernel_times synchronises on the last
+ * forward and writes up to `cap` durations in ms (order: pool, compressed +
+ * top-k, selection, epilogue, special, special-merge) and their
+ * names (static strings).  Returns the number of entries or a negative
+ * status. */
+GSA_API int gsa_set_profiling(gsa_ctx *ctx, int enable);
+GSA_API int gsa_get_kernel_times(gsa_ctx *ctx, float *ms, const char **names, int cap);
+
+/* Synchronise the context's last stream and return (then clear) the device
+ * error word: GSA_OK, GSA_ERR_DEVICE_BOUNDS or GSA_ERR_DEVICE_TIMEOUT. */
+GSA_API int gsa_get_status(gsa_ctx *ctx);
+
+/* Static text for a status code. */
+GSA_API const char *gsa_strerror(int code);
+
+/* Free the workspace and the context; NULL is accepted. */
+GSA_API void gsa_destroy(gsa_ctx *ctx);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GSA_B200_H */

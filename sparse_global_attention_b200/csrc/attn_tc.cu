@@ -1,0 +1,554 @@
+// Attention on 5th-generation tensor cores (tcgen05 + TMEM + TMA), shared by
+//   K2  compressed branch with the fused streaming top-k of S_guide
+//       ("Speed3R: Sparse Feed-forward 3D Reconstruction Models", Paper-Notes
+//       CVPR 2026, compression branch; "高效 Triton Kernel 实现": top-k kept
+//       while the FlashAttention loop runs, S_guide never materialised);
+//   K5  special tokens over every token (split over key ranges, merged later);
+//   K6  dense global attention (the comparison baseline).
+//
+// One CTA owns two 128-row query tiles (M = 256) that share every K/V tile, so
+// each key byte crosses L2 -> SM once per 256 queries.  Warp roles:
+//   warps 0-3  softmax for query tile 0 (thread = row = TMEM lane)
+//   warps 4-7  softmax for query tile 1
+//   warp  8    TMA producer: Q tiles once, then K/V tiles into a 3-stage ring
+//   warp  9    MMA issuer (one thread): S_i = Q_i K^T (SS form, both operands
+//              in 128B-swizzled shared memory) and O_i += P_i V (TS form: P_i
+//              read from TMEM, V as an MN-major shared-memory operand)
+// TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,320), O_1 [320,384).
+// Softmax threads read their row of S_i, write P_i (bf16 pairs) back over the
+// first 64 columns of S_i, and rescale O_i in TMEM only when the running max
+// grows by more than 2^8 (lazy rescaling: the stale max keeps every
+// exponent <= 2^8, and numerator and denominator share it).
+//
+// Guide scores (K2): Q and K arrive as bf16 pairs hi + lo (lo = bf16 of the
+// residual), S = Qhi Khi^T + Qhi Klo^T + Qlo Khi^T, accurate to ~2^-17 of
+// |q||k|, so the top-k agrees with exact scores wherever the k-th and
+// (k+1)-th scores differ by more than a few 1e-5 relative.  The streaming
+// top-k is a sorted register list per thread (its row): a score strictly
+// greater than the current k-th enters by an unrolled shift network; keys
+// arrive in increasing region order, so on equal scores the lower region
+// stays ahead, as the tie rule requires.
+//
+// All mbarrier waits are bounded by the global timer; a wait that runs out
+// records GSA_ERR_DEVICE_TIMEOUT and the CTA drains and exits.
+#include <cuda.h>
+
+#include "gsa_kernels.h"
+#include "tc_ptx.cuh"
+
+namespace gsa {
+
+namespace {
+
+using namespace tc;
+
+constexpr int TBM = 128;                 // rows per query tile
+constexpr int TBN = 128;                 // keys per tile
+constexpr int TILE = TBN * 128;          // bytes of one 128x64 bf16 tile
+constexpr int NST = 3;                   // K/V ring depth
+constexpr int NTHREADS = 320;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr float RESCALE_LOG2 = 8.f;      // rescale O when the max grows by > 2^8
+
+constexpr uint32_t IDESC_QK = idesc_bf16(128, 128, false);
+constexpr uint32_t IDESC_PV = idesc_bf16(128, 64, true);
+
+template <int KC>
+struct Lay {
+  static constexpr bool TOPK = KC > 0;
+  static constexpr int QT = TOPK ? 2 : 1;              // tiles per query tile (hi[, lo])
+  static constexpr int KT = TOPK ? 3 : 2;              // tiles per stage: K hi, [K lo], V
+  static constexpr int KV = 2 * QT * TILE;             // Q_i hi at i*TILE, lo at (2+i)*TILE
+  static constexpr int STAGE = KT * TILE;
+  static constexpr int BAR = KV + NST * STAGE;
+  // barriers: q_full, full[NST], empty[NST], s_full[2], p_full[2], pv_done[2], fin
+  static constexpr int NBAR = 1 + 2 * NST + 6 + 1;
+  static constexpr int TMEM_SLOT = BAR + NBAR * 8;
+  static constexpr int BYTES = TMEM_SLOT + 16 + 1024;   // + alignment slack
+};
+
+struct Bars {
+  uint32_t base;
+  __device__ uint32_t q_full() const { return base; }
+  __device__ uint32_t full(int s) const { return base + 8 * (1 + s); }
+  __device__ uint32_t empty(int s) const { return base + 8 * (1 + NST + s); }
+  __device__ uint32_t s_full(int i) const { return base + 8 * (1 + 2 * NST + i); }
+  __device__ uint32_t p_full(int i) const { return base + 8 * (3 + 2 * NST + i); }
+  __device__ uint32_t pv_done(int i) const { return base + 8 * (5 + 2 * NST + i); }
+  __device__ uint32_t fin() const { return base + 8 * (7 + 2 * NST); }
+};
+
+__device__ __forceinline__ int tile_seg(const AttnArgs& a, int tt, long long& kb) {
+  const int seg = (a.nseg > 1 && tt >= a.tiles0) ? 1 : 0;
+  kb = static_cast<long long>(seg ? tt - a.tiles0 : tt) * TBN;
+  return seg;
+}
+
+
+// validity bits of 32 consecutive keys starting at key0 (bit e = key0 + e)
+__device__ __noinline__ uint32_t chunk_valid(int km, Grid g, int nk, long long key0) {
+  const long long lim = nk - key0;
+  uint32_t m = lim >= 32 ? ~0u : (lim <= 0 ? 0u : ((1u << lim) - 1u));
+  if (km != MASK_NONE) {
+    for (int e = 0; e < 32; ++e)
+      if (((m >> e) & 1u) && !key_valid(km, g, key0 + e)) m &= ~(1u << e);
+  }
+  return m;
+}
+
+__device__ __forceinline__ void apply_mask(uint32_t* v, uint32_t msk) {
+#pragma unroll
+  for (int e = 0; e < 32; ++e) v[e] = ((msk >> e) & 1u) ? v[e] : 0xff800000u;   // -inf
+}
+
+__device__ __forceinline__ bool is_fixed_region(const AttnArgs& a, int col) {
+  const int fr = col / a.rpf;
+  bool hit = false;
+  for (int f = 0; f < a.n_fixed; ++f) hit = hit || (a.fixed[f] == fr);
+  return hit;
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16};\n" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+// Lazy rescale: move the reference max only when the row max grew by more than
+// 2^8; O_i (in TMEM) is rescaled once PV of the previous tile has completed.
+// The decision to touch TMEM is warp-uniform (TMEM loads are warp-collective).
+__device__ __forceinline__ void rescale(float mx, float& m, float& l, int j, int qi, uint32_t tO,
+                                        const Bars& bars, int* err, bool& ok, float sl2) {
+  const float m_new = fmaxf(m, mx);
+  const bool need = (m == -INFINITY) ? (m_new != -INFINITY) : ((m_new - m) * sl2 > RESCALE_LOG2);
+  float alpha = 1.f;
+  if (need) {
+    alpha = (m == -INFINITY) ? 0.f : ex2((m - m_new) * sl2);
+    m = m_new;
+  }
+  l *= alpha;
+  if (__any_sync(0xffffffffu, need && alpha != 0.f) && j > 0) {
+    ok = __all_sync(0xffffffffu, mbar_wait(bars.pv_done(qi), (j - 1) & 1, err));
+    if (!ok) return;
+    tc_fence_after();
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      uint32_t v[32];
+      tmem_ld32(tO + 32 * c, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+      tmem_st32(tO + 32 * c, v);
+    }
+    tmem_wait_st();
+  }
+}
+
+template <int KC>
+__device__ __forceinline__ void topk_insert(float (&ts)[KC > 0 ? KC : 1], int (&ti)[KC > 0 ? KC : 1],
+                                            float s, int id) {
+  bool h = s > ts[KC - 1];
+#pragma unroll
+  for (int p = KC - 1; p > 0; --p) {
+    const bool g = s > ts[p - 1];
+    ts[p] = g ? ts[p - 1] : (h ? s : ts[p]);
+    ti[p] = g ? ti[p - 1] : (h ? id : ti[p]);
+    h = g;
+  }
+  if (h) {
+    ts[0] = s;
+    ti[0] = id;
+  }
+}
+
+template <int KC>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qlo,
+                   const __grid_constant__ CUtensorMap tm_k0, const __grid_constant__ CUtensorMap tm_v0,
+                   const __grid_constant__ CUtensorMap tm_k1, const __grid_constant__ CUtensorMap tm_v1,
+                   const __grid_constant__ CUtensorMap tm_klo, const AttnArgs a) {
+  using L = Lay<KC>;
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte alignment for the 128B-swizzle atoms
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - raw);
+  const Bars bars{sbase + L::BAR};
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sgen + L::TMEM_SLOT);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.z, split = blockIdx.y;
+  const int row0 = blockIdx.x * (2 * TBM);
+  const int t_begin = split * a.tiles_per_split;
+  const int t_end = min(t_begin + a.tiles_per_split, a.tiles_total);
+  const int ntile = max(t_end - t_begin, 0);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bars.q_full(), 1);
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(bars.full(s), 1);
+      mbar_init(bars.empty(s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bars.s_full(i), 1);
+      mbar_init(bars.p_full(i), TBM);
+      mbar_init(bars.pv_done(i), 1);
+    }
+    mbar_init(bars.fin(), 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc<TMEM_COLS>(smem_u32(tmem_slot));
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && ntile > 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k0);
+      prefetch_tmap(&tm_v0);
+      const int qy = h * a.n_q + row0;
+      mbar_expect_tx(bars.q_full(), 2 * L::QT * TILE);
+      tma_load_2d(sbase + 0 * TILE, &tm_q, 0, qy, bars.q_full());
+      tma_load_2d(sbase + 1 * TILE, &tm_q, 0, qy + TBM, bars.q_full());
+      if constexpr (L::TOPK) {
+        tma_load_2d(sbase + 2 * TILE, &tm_qlo, 0, qy, bars.q_full());
+        tma_load_2d(sbase + 3 * TILE, &tm_qlo, 0, qy + TBM, bars.q_full());
+      }
+      int issued = 0;
+      for (int it = 0; it < ntile; ++it) {
+        const int s = it % NST;
+        if (it >= NST && !mbar_wait(bars.empty(s), ((it / NST) - 1) & 1, a.err)) break;
+        long long kb;
+        const int seg = tile_seg(a, t_begin + it, kb);
+        const int y = static_cast<int>(static_cast<long long>(h) * a.n_k[seg] + kb);
+        const uint32_t st = sbase + L::KV + s * L::STAGE;
+        mbar_expect_tx(bars.full(s), L::KT * TILE);
+        tma_load_2d(st, seg ? &tm_k1 : &tm_k0, 0, y, bars.full(s));
+        if constexpr (L::TOPK) tma_load_2d(st + TILE, &tm_klo, 0, y, bars.full(s));
+        tma_load_2d(st + (L::KT - 1) * TILE, seg ? &tm_v1 : &tm_v0, 0, y, bars.full(s));
+        ++issued;
+      }
+      // drain: every issued copy has landed before the CTA may exit
+      for (int it = max(0, issued - NST); it < issued; ++it)
+        mbar_wait(bars.full(it % NST), (it / NST) & 1, a.err);
+      mbar_wait(bars.q_full(), 0, a.err);
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && ntile > 0) {
+      bool ok = mbar_wait(bars.q_full(), 0, a.err);
+      tc_fence_after();
+      for (int j = 0; ok && j <= ntile; ++j) {
+        if (j < ntile) {
+          ok = mbar_wait(bars.full(j % NST), (j / NST) & 1, a.err);
+          if (!ok) break;
+          tc_fence_after();
+        }
+        for (int i = 0; i < 2 && ok; ++i) {
+          if (j > 0) {
+            // O_i += P_{i,j-1} V_{j-1}
+            ok = mbar_wait(bars.p_full(i), (j - 1) & 1, a.err);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t vs = sbase + L::KV + ((j - 1) % NST) * L::STAGE + (L::KT - 1) * TILE;
+#pragma unroll
+            for (int ks = 0; ks < TBN / 16; ++ks) {
+              const uint64_t bd = sdesc_sw128(vs + ks * 2048, 8192, 1024);
+              asm volatile(
+                  "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], "
+                  "[%1], %2, %3, p;\n}\n" ::"r"(tmem + 256 + 64 * i),
+                  "r"(tmem + 128 * i + 8 * ks), "l"(bd), "r"(IDESC_PV), "r"((j > 1 || ks > 0) ? 1u : 0u)
+                  : "memory");
+            }
+            mma_commit(bars.pv_done(i));
+          }
+          if (j < ntile) {
+            // S_{i,j} = Q_i K_j^T (guide: + Q_i^hi K_j^lo + Q_i^lo K_j^hi)
+            const uint32_t ks0 = sbase + L::KV + (j % NST) * L::STAGE;
+            const uint32_t qs = sbase + i * TILE;
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              const uint64_t ad = sdesc_sw128(qs + 32 * ks, 16, 1024);
+              const uint64_t bd = sdesc_sw128(ks0 + 32 * ks, 16, 1024);
+              mma_bf16_ss(tmem + 128 * i, ad, bd, IDESC_QK, ks > 0 ? 1u : 0u);
+              if constexpr (L::TOPK) {
+                const uint64_t bl = sdesc_sw128(ks0 + TILE + 32 * ks, 16, 1024);
+                const uint64_t al = sdesc_sw128(qs + 2 * TILE + 32 * ks, 16, 1024);
+                mma_bf16_ss(tmem + 128 * i, ad, bl, IDESC_QK, 1u);
+                mma_bf16_ss(tmem + 128 * i, al, bd, IDESC_QK, 1u);
+              }
+            }
+            mma_commit(bars.s_full(i));
+          }
+        }
+        if (ok && j > 0) mma_commit(bars.empty((j - 1) % NST));
+      }
+      mma_commit(bars.fin());
+      mbar_wait(bars.fin(), 0, a.err);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int qi = warp >> 2;                         // query tile 0 or 1
+    const int r = threadIdx.x & 127;                  // row in the tile = TMEM lane
+    const int row = row0 + qi * TBM + r;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + 128 * qi;
+    const uint32_t tO = tmem + lane_off + 256 + 64 * qi;
+    const float sl2 = a.scale_log2;
+    float m = -INFINITY, l = 0.f;
+    float ts[KC > 0 ? KC : 1], thr = -INFINITY;
+    int ti[KC > 0 ? KC : 1];
+#pragma unroll
+    for (int p = 0; p < (KC > 0 ? KC : 1); ++p) {
+      ts[p] = -INFINITY;
+      ti[p] = -1;
+    }
+    bool ok = true;
+    for (int j = 0; j < ntile; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bars.s_full(qi), j & 1, a.err));
+      if (!ok) break;
+      tc_fence_after();
+      long long kb;
+      const int seg = tile_seg(a, t_begin + j, kb);
+      const int nk = a.n_k[seg];
+      const int km = a.kmask[seg];
+      // key validity of the tile's four 32-key chunks (all ones unless ragged or padded)
+      uint32_t vm[4] = {~0u, ~0u, ~0u, ~0u};
+      if (km != MASK_NONE || kb + TBN > nk) {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) vm[c] = chunk_valid(km, a.g, nk, kb + 32 * c);
+      }
+      float mx = -INFINITY;
+      if constexpr (!L::TOPK) {
+        // whole row of S in registers: one TMEM wait per tile
+        uint32_t v[128];
+        tmem_ld64(tS, v);
+        tmem_ld64(tS + 64, v + 64);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (vm[c] != ~0u) apply_mask(v + 32 * c, vm[c]);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(v[32 * c + e]));
+        }
+        rescale(mx, m, l, j, qi, tO, bars, a.err, ok, sl2);
+        if (!ok) break;
+        const float mb = (m == -INFINITY) ? 0.f : m * sl2;
+        float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float p0 = ex2(fmaf(__uint_as_float(v[32 * c + e]), sl2, -mb));
+            const float p1 = ex2(fmaf(__uint_as_float(v[32 * c + e + 1]), sl2, -mb));
+            l0 += p0;
+            l1 += p1;
+            pk[e >> 1] = pack_bf16(p0, p1);
+          }
+          tmem_st16(tS + 16 * c, pk);
+        }
+        l += l0 + l1;
+      } else {
+        // pass 1, two 64-key halves: row max and the streaming top-k
+#pragma unroll 1
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t v[64];
+          tmem_ld64(tS + 64 * hf, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const uint32_t msk = vm[2 * hf + c];
+            if (msk != ~0u) apply_mask(v + 32 * c, msk);
+            uint32_t cb = 0;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float x = __uint_as_float(v[32 * c + e]);
+              mx = fmaxf(mx, x);
+              cb |= (x > thr ? 1u : 0u) << e;
+            }
+            // rare: a score beats the current k-th; take the candidates in column order
+            while (cb) {
+              const int e = __ffs(cb) - 1;
+              cb &= cb - 1;
+              float x = __uint_as_float(v[32 * c]);
+#pragma unroll
+              for (int q = 1; q < 32; ++q)
+                if (q == e) x = __uint_as_float(v[32 * c + q]);
+              if (!(x > thr)) continue;
+              const int col = static_cast<int>(kb) + 64 * hf + 32 * c + e;
+              if (a.n_fixed && is_fixed_region(a, col)) continue;
+              topk_insert<KC>(ts, ti, x, col);
+              float t = ts[KC - 1];
+#pragma unroll
+              for (int p = 0; p < KC; ++p)
+                if (p == a.kc - 1) t = ts[p];
+              thr = t;
+            }
+          }
+        }
+        rescale(mx, m, l, j, qi, tO, bars, a.err, ok, sl2);
+        if (!ok) break;
+        // pass 2: P = exp2((S - m) * scale * log2e) as bf16 pairs over S's first 64 columns
+        const float mb = (m == -INFINITY) ? 0.f : m * sl2;
+        float l0 = 0.f, l1 = 0.f;
+#pragma unroll 1
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t v[64];
+          tmem_ld64(tS + 64 * hf, v);
+          tmem_wait_ld();
+          if (vm[2 * hf] != ~0u) apply_mask(v, vm[2 * hf]);
+          if (vm[2 * hf + 1] != ~0u) apply_mask(v + 32, vm[2 * hf + 1]);
+          uint32_t pk[32];
+#pragma unroll
+          for (int e = 0; e < 64; e += 2) {
+            const float p0 = ex2(fmaf(__uint_as_float(v[e]), sl2, -mb));
+            const float p1 = ex2(fmaf(__uint_as_float(v[e + 1]), sl2, -mb));
+            l0 += p0;
+            l1 += p1;
+            pk[e >> 1] = pack_bf16(p0, p1);
+          }
+          tmem_st32(tS + 32 * hf, pk);
+        }
+        l += l0 + l1;
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bars.p_full(qi));
+    }
+    // ---- epilogue: O_i row from TMEM ----------------------------------------
+    if (ok && ntile > 0) ok = mbar_wait(bars.pv_done(qi), (ntile - 1) & 1, a.err);
+    ok = __all_sync(0xffffffffu, ok);
+    tc_fence_after();
+    float o[64];
+    if (ok && ntile > 0) {
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tO + 32 * c, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[32 * c + e] = __uint_as_float(v[e]);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 64; ++e) o[e] = 0.f;
+    }
+    if (row < a.n_q) {
+      if (a.n_split == 1) {
+        float inv = l > 0.f ? 1.f / l : 0.f;
+        if (a.q_mask != MASK_NONE && !key_valid(a.q_mask, a.g, row)) inv = 0.f;
+        const long long base = h * a.o_hs + static_cast<long long>(row) * D;
+        if (a.o16) {
+#pragma unroll
+          for (int e = 0; e < 64; e += 8) {
+            const uint4 w = make_uint4(pack_bf16(o[e] * inv, o[e + 1] * inv), pack_bf16(o[e + 2] * inv, o[e + 3] * inv),
+                                       pack_bf16(o[e + 4] * inv, o[e + 5] * inv), pack_bf16(o[e + 6] * inv, o[e + 7] * inv));
+            *reinterpret_cast<uint4*>(a.o16 + base + e) = w;
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 64; e += 4)
+            *reinterpret_cast<float4*>(a.o32 + base + e) =
+                make_float4(o[e] * inv, o[e + 1] * inv, o[e + 2] * inv, o[e + 3] * inv);
+        }
+      } else {
+        const long long pr = (static_cast<long long>(split) * a.H + h) * a.n_q + row;
+#pragma unroll
+        for (int e = 0; e < 64; e += 4)
+          *reinterpret_cast<float4*>(a.part_o + pr * D + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+        *reinterpret_cast<float2*>(a.part_ml + pr * 2) = make_float2(m, l);
+      }
+      if constexpr (L::TOPK) {
+        const long long base = (static_cast<long long>(h) * a.n_q + row) * a.kc;
+#pragma unroll
+        for (int p = 0; p < KC; ++p) {
+          if (p < a.kc) {
+            a.cand[base + p] = ti[p];
+            if (a.cand_user) a.cand_user[base + p] = ti[p];
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc<TMEM_COLS>(tmem);
+}
+
+// ---- tensor maps ----------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2D bf16 tensor [rows][64] with 128-row, 128B-swizzled boxes
+bool make_map(CUtensorMap* m, const void* base, long long rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || !base || rows <= 0 || rows > 0x7fffffffLL) return false;
+  const cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {128};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int KC>
+cudaError_t launch_kc(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t st) {
+  const int sm = Lay<KC>::BYTES;
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<KC>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+  if (e != cudaSuccess) return e;
+  dim3 grid((a.n_q + 2 * TBM - 1) / (2 * TBM), a.n_split, a.H);
+  attn_tc_kernel<KC><<<grid, NTHREADS, sm, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int attn_tc_tiles(long long n) { return static_cast<int>((n + TBN - 1) / TBN); }
+
+cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
+  CUtensorMap maps[7];
+  memset(maps, 0, sizeof(maps));
+  const long long H = a.H;
+  if (!make_map(&maps[0], a.q, H * a.n_q)) return cudaErrorInvalidValue;
+  maps[1] = maps[0];
+  if (a.kc > 0 && !make_map(&maps[1], a.q_lo, H * a.n_q)) return cudaErrorInvalidValue;
+  if (!make_map(&maps[2], a.k[0], H * a.n_k[0]) || !make_map(&maps[3], a.v[0], H * a.n_k[0]))
+    return cudaErrorInvalidValue;
+  maps[4] = maps[2];
+  maps[5] = maps[3];
+  if (a.nseg > 1 && (!make_map(&maps[4], a.k[1], H * a.n_k[1]) || !make_map(&maps[5], a.v[1], H * a.n_k[1])))
+    return cudaErrorInvalidValue;
+  maps[6] = maps[2];
+  if (a.kc > 0 && !make_map(&maps[6], a.k_lo, H * a.n_k[0])) return cudaErrorInvalidValue;
+  if (a.kc == 0) return launch_kc<0>(a, maps, st);
+  if (a.kc <= 8) return launch_kc<8>(a, maps, st);
+  if (a.kc <= 16) return launch_kc<16>(a, maps, st);
+  if (a.kc <= 32) return launch_kc<32>(a, maps, st);
+  if (a.kc <= 64) return launch_kc<64>(a, maps, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace gsa

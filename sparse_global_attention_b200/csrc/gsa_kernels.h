@@ -1,0 +1,114 @@
+// Host-side launch interface of the GSA kernels (internal to the library).
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "gsa_common.cuh"
+
+namespace gsa {
+
+// ---- K1 pool ---------------------------------------------------------------
+struct PoolArgs {
+  const void* src[3];        // Q/K/V image tokens [H][F][Hp][Wp][64]
+  __nv_bfloat16* out16[3];   // pooled, bf16 (round to nearest) [H][R][64]  (nullptr = skip)
+  __nv_bfloat16* outlo[3];   // pooled minus its bf16 value, in bf16         (nullptr = skip)
+  float* out32[3];           // pooled, fp32 [H][R][64]                      (nullptr = skip)
+  int H, F, Hp, Wp, Hv, Wv, s;
+};
+cudaError_t launch_pool(const PoolArgs& a, bool fp32, cudaStream_t st);
+
+// ---- attention core (K2 compressed + top-k, K5 special, K6 dense) ----------
+struct AttnArgs {
+  const __nv_bfloat16* q;    // [H][n_q][64]
+  const __nv_bfloat16* q_lo; // top-k only: low bf16 parts of q and k[0]
+  const __nv_bfloat16* k_lo;
+  long long q_hs;            // head stride (elements)
+  int n_q;                   // query rows per head
+  int q_mask;                // MASK_NONE or MASK_DENSE: pad query rows output 0
+  int nseg;                  // 1 or 2 key segments, tiled separately
+  const __nv_bfloat16* k[2];
+  const __nv_bfloat16* v[2];
+  long long kv_hs[2];
+  int n_k[2];
+  int kmask[2];              // MaskMode per segment
+  int tiles0;                // 64-key tiles of segment 0
+  int tiles_total;
+  int tiles_per_split;
+  int n_split;               // 1 = write final output, >1 = write partials
+  int H;
+  Grid g;
+  float scale_log2;          // softmax scale * log2(e)
+  __nv_bfloat16* o16;        // final output [H][n_q][64] (one of o16/o32)
+  float* o32;
+  long long o_hs;
+  float* part_o;             // [n_split][H][n_q][64] unnormalised
+  float* part_ml;            // [n_split][H][n_q][2]  (running max in raw score units, sum)
+  // streaming top-k of the raw scores (compressed branch only)
+  int kc;                    // regions kept per row (the top-k)
+  int* cand;                 // [H][n_q][kc] region indices, best first
+  int* cand_user;            // optional copy for the caller
+  int rpf;                   // regions per frame
+  int n_fixed;
+  int fixed[MAX_FIXED];      // frames excluded from the candidates
+  int* err;                  // device error word
+};
+cudaError_t launch_attn(const AttnArgs& a, bool topk, cudaStream_t st);
+// tcgen05/TMEM/TMA version: 2 x 128 query rows per CTA, 128-key tiles; the
+// top-k runs when a.kc > 0 (a.q_lo / a.k_lo required)
+cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st);
+int attn_tc_tiles(long long n);
+
+struct MergeArgs {
+  const float* part_o;
+  const float* part_ml;
+  int n_split, H, n_q;
+  float scale_log2;
+  __nv_bfloat16* o16;
+  float* o32;
+  long long o_hs;
+};
+cudaError_t launch_merge(const MergeArgs& a, cudaStream_t st);
+
+// ---- K3 selection ----------------------------------------------------------
+struct SelArgs {
+  const void* q_img;         // [H][F][Hp][Wp][64]
+  const void* k_img;
+  const void* v_img;
+  const void* k_spec;        // [H][F][ns][64]
+  const void* v_spec;
+  const int* idx;            // [H][R][topk]
+  void* o_sel;               // [H][F][Hp][Wp][64]
+  int H, F, R, rpf, topk, s;
+  Grid g;
+  float scale_log2;
+  int n_fixed;
+  int fixed[MAX_FIXED];
+  int* err;
+};
+cudaError_t launch_sel(const SelArgs& a, bool fp32, cudaStream_t st);
+
+// ---- K4 upsample + gate + blend --------------------------------------------
+struct EpiArgs {
+  const void* q_img;         // [H][F][Hp][Wp][64]
+  const void* o_sel;         // [H][F][Hp][Wp][64]
+  const float* o_comp;       // [H][R][64] fp32
+  const void* w_g;           // [H][64][64]
+  void* o_img;               // [H][F][Hp][Wp][64]
+  int H, F, R, rpf, s;
+  Grid g;
+  int gate_mode;
+};
+cudaError_t launch_epilogue(const EpiArgs& a, bool fp32, cudaStream_t st);
+
+// ---- fp32 (SIMT) variants for fp32 contexts ---------------------------------
+struct AttnF32Args {
+  const float* q; long long q_hs; int n_q; int q_mask;
+  int nseg;
+  const float* k[2]; const float* v[2]; long long kv_hs[2]; int n_k[2]; int kmask[2];
+  int H; Grid g; float scale;
+  float* o; long long o_hs;
+  int kc; int* cand; int* cand_user; int rpf; int n_fixed; int fixed[MAX_FIXED];
+};
+cudaError_t launch_attn_f32(const AttnF32Args& a, bool topk, cudaStream_t st);
+
+}  // namespace gsa

@@ -1,0 +1,351 @@
+// K3: selection-branch attention.
+//
+// "Speed3R: Sparse Feed-forward 3D Reconstruction Models" (Paper-Notes,
+// CVPR 2026), selection branch: for each compressed query the top-k regions
+// are chosen from S_guide, their full-resolution K/V tokens are gathered, and
+// O_sel = Attention(Q_img, K_sel, V_sel); the queries of one compression
+// window share one KV set.  For the VGGT adaptation ("Speed3R-VGGT 适配") the
+// key set also holds a fixed global context: every token of the reference
+// frame and of the frames sampled every 100 frames.
+//
+// bf16 path: one warp per window (s*s <= 16 queries fill one m16 MMA tile);
+// 4 windows per CTA, neighbours in raster order so their overlapping region
+// choices meet in L2.  Each warp gathers its keys 32 at a time (the tokens of
+// the selected regions, then the fixed context) into its own double-buffered
+// shared-memory stage with 16-byte cp.async, and runs S = Q K^T, an online
+// softmax and O += P V on m16n8k16 MMAs.  Pad keys are masked, pad queries
+// write 0.
+//
+// fp32 path: one thread per query token with fp32 FMA (tiny configs).
+#include "gsa_common.cuh"
+#include "gsa_kernels.h"
+
+namespace gsa {
+
+namespace {
+
+constexpr int SEL_BN = 32;                     // keys per stage
+constexpr int SEL_TILE = SEL_BN * 128;         // bytes of one K (or V) stage
+constexpr int SEL_WARP_SMEM = (16 * 128 + 2 * 2 * SEL_TILE + KC_MAX * 8 + 2 * SEL_BN + 127) / 128 * 128;
+constexpr int SEL_WARPS = 4;
+
+// Geometry of one selected region: .x = flat token index (within the head) of
+// its top-left token, .y = (valid rows << 16) | valid cols, both capped at S.
+template <int S>
+__device__ __forceinline__ int2 region_base(const SelArgs& a, int reg) {
+  const int f = reg / a.rpf, rr = reg - f * a.rpf;
+  const int rx = a.g.Wp / S;
+  const int i = rr / rx, j = rr - i * rx;
+  const int ly = min(a.g.Hv - i * S, S), lx = min(a.g.Wv - j * S, S);
+  return make_int2((f * a.g.Hp + i * S) * a.g.Wp + j * S, (ly << 16) | lx);
+}
+
+// Source of key position p of a window's key list: the s*s tokens of each
+// selected region in order (regions described by `rb`), then per fixed frame
+// its special tokens and its padded image grid.  Returns false for pad tokens
+// and positions past the end.
+template <int S>
+__device__ __forceinline__ bool key_src(const SelArgs& a, const int2* rb, int p, int nk_dyn,
+                                        int nkeys, long long& off, bool& spec) {
+  spec = false;
+  off = 0;
+  if (p < nk_dyn) {
+    const int slot = p / (S * S), tq = p % (S * S);
+    const int2 r = rb[slot];
+    const int dy = tq / S, dx = tq % S;
+    off = r.x + dy * a.g.Wp + dx;
+    return dy < (r.y >> 16) && dx < (r.y & 0xffff);
+  }
+  if (p >= nkeys) return false;
+  const int per = a.g.ns + a.g.Hp * a.g.Wp;
+  const int pf = p - nk_dyn;
+  const int fi = pf / per, o = pf - fi * per;
+  int frame = 0;
+  for (int i = 0; i < a.n_fixed; ++i)
+    if (i == fi) frame = a.fixed[i];
+  if (o < a.g.ns) {
+    spec = true;
+    off = static_cast<long long>(frame) * a.g.ns + o;
+    return true;
+  }
+  off = static_cast<long long>(frame) * a.g.Hp * a.g.Wp + (o - a.g.ns);
+  return a.g.img_valid(o - a.g.ns);
+}
+
+template <int S>
+__global__ void __launch_bounds__(SEL_WARPS * 32) sel_kernel_bf16(const SelArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3, mi = lane >> 3, lr = lane & 7;
+  uint8_t* wbase = smem + warp * SEL_WARP_SMEM;
+  const uint32_t sQ = smem_u32(wbase);
+  const uint32_t sKV = sQ + 16 * 128;
+  int2* sReg = reinterpret_cast<int2*>(wbase + 16 * 128 + 4 * SEL_TILE);
+  uint8_t* sValid = reinterpret_cast<uint8_t*>(sReg + KC_MAX);
+
+  const long long win = static_cast<long long>(blockIdx.x) * SEL_WARPS + warp;
+  if (win >= static_cast<long long>(a.H) * a.R) return;      // warp-uniform
+  const int h = static_cast<int>(win / a.R);
+  const int r = static_cast<int>(win - static_cast<long long>(h) * a.R);
+  const long long img_hs = static_cast<long long>(a.F) * a.g.Hp * a.g.Wp * D;
+  const long long spec_hs = static_cast<long long>(a.F) * a.g.ns * D;
+  const __nv_bfloat16* qh = reinterpret_cast<const __nv_bfloat16*>(a.q_img) + h * img_hs;
+  const __nv_bfloat16* kh = reinterpret_cast<const __nv_bfloat16*>(a.k_img) + h * img_hs;
+  const __nv_bfloat16* vh = reinterpret_cast<const __nv_bfloat16*>(a.v_img) + h * img_hs;
+  const __nv_bfloat16* ksh = reinterpret_cast<const __nv_bfloat16*>(a.k_spec) + h * spec_hs;
+  const __nv_bfloat16* vsh = reinterpret_cast<const __nv_bfloat16*>(a.v_spec) + h * spec_hs;
+
+  // window geometry
+  const int f = r / a.rpf, rr0 = r - f * a.rpf;
+  const int rx = a.g.Wp / S;
+  const int wi = rr0 / rx, wj = rr0 - wi * rx;
+
+  // selected regions of this window
+  for (int j = lane; j < a.topk; j += 32) {
+    int v = a.idx[win * a.topk + j];
+    if (v < 0 || v >= a.R) {
+      set_error(a.err, ERR_BOUNDS);
+      v = 0;
+    }
+    sReg[j] = region_base<S>(a, v);
+  }
+  // queries: token q = (a_, b_) of the window, rows >= s*s are zero
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int e = lane + 32 * it;
+    const int row = e >> 3, c = e & 7;
+    const int y = wi * S + row / S, x = wj * S + row % S;
+    const bool ok = row < S * S && y < a.g.Hv && x < a.g.Wv;
+    const long long tok = ok ? (static_cast<long long>(f) * a.g.Hp + y) * a.g.Wp + x : 0;
+    cp_async16(sQ + swz(row, c), qh + tok * D + c * 8, ok ? 16 : 0);
+  }
+  cp_async_commit();
+  __syncwarp();
+
+  const int nk_dyn = a.topk * S * S;
+  const int nkeys = nk_dyn + a.n_fixed * (a.g.ns + a.g.Hp * a.g.Wp);
+  const int nblk = (nkeys + SEL_BN - 1) / SEL_BN;
+
+  auto issue = [&](int blk, int st) {
+    const uint32_t sK = sKV + st * 2 * SEL_TILE;
+    const uint32_t sV = sK + SEL_TILE;
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int e = lane + 32 * it;
+      const int key = e >> 3, c = e & 7;
+      long long off;
+      bool spec;
+      const bool ok = key_src<S>(a, sReg, blk * SEL_BN + key, nk_dyn, nkeys, off, spec);
+      const __nv_bfloat16* kp = (spec ? ksh : kh) + off * D + c * 8;
+      const __nv_bfloat16* vp = (spec ? vsh : vh) + off * D + c * 8;
+      cp_async16(sK + swz(key, c), ok ? kp : kh, ok ? 16 : 0);
+      cp_async16(sV + swz(key, c), ok ? vp : vh, ok ? 16 : 0);
+      if (c == 0) sValid[st * SEL_BN + key] = ok ? 1 : 0;
+    }
+  };
+
+  issue(0, 0);
+  cp_async_commit();
+  cp_async_wait<1>();
+  __syncwarp();
+  uint32_t qf[4][4];
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks)
+    ldsm_x4(sQ + swz(lr + 8 * (mi & 1), 2 * ks + (mi >> 1)), qf[ks][0], qf[ks][1], qf[ks][2],
+            qf[ks][3]);
+
+  float o[8][4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  float m[2] = {-INFINITY, -INFINITY};
+  float l[2] = {0.f, 0.f};
+  const float sl2 = a.scale_log2;
+
+  for (int blk = 0; blk < nblk; ++blk) {
+    const int st = blk & 1;
+    __syncwarp();
+    if (blk + 1 < nblk) issue(blk + 1, st ^ 1);
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncwarp();
+    const uint32_t sK = sKV + st * 2 * SEL_TILE;
+    const uint32_t sV = sK + SEL_TILE;
+
+    float s[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+      for (int np = 0; np < 2; ++np) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(sK + swz(16 * np + lr + 8 * (mi >> 1), 2 * ks + (mi & 1)), b0, b1, b2, b3);
+        mma_bf16(s[2 * np], qf[ks], b0, b1);
+        mma_bf16(s[2 * np + 1], qf[ks], b2, b3);
+      }
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e)
+        if (!sValid[st * SEL_BN + 8 * nt + 2 * t + e]) {
+          s[nt][e] = -INFINITY;
+          s[nt][2 + e] = -INFINITY;
+        }
+
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      float mx = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) mx = fmaxf(mx, fmaxf(s[nt][2 * rr], s[nt][2 * rr + 1]));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const float m_new = fmaxf(m[rr], mx);
+      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+      const float alpha = ex2((m[rr] - m_use) * sl2);
+      l[rr] *= alpha;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        o[nt][2 * rr] *= alpha;
+        o[nt][2 * rr + 1] *= alpha;
+      }
+      const float mb = m_use * sl2;
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
+        const float p0 = ex2(fmaf(s[nt][2 * rr], sl2, -mb));
+        const float p1 = ex2(fmaf(s[nt][2 * rr + 1], sl2, -mb));
+        s[nt][2 * rr] = p0;
+        s[nt][2 * rr + 1] = p1;
+        l[rr] += p0 + p1;
+      }
+      m[rr] = m_new;
+    }
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk) {
+      uint32_t pa[4];
+      pa[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
+      pa[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
+      pa[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+      pa[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+#pragma unroll
+      for (int dp = 0; dp < 4; ++dp) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(sV + swz(16 * kk + lr + 8 * (mi & 1), 2 * dp + (mi >> 1)), b0, b1, b2, b3);
+        mma_bf16(o[2 * dp], pa, b0, b1);
+        mma_bf16(o[2 * dp + 1], pa, b2, b3);
+      }
+    }
+  }
+  cp_async_wait<0>();
+
+  __nv_bfloat16* oh = reinterpret_cast<__nv_bfloat16*>(a.o_sel) + h * img_hs;
+#pragma unroll
+  for (int rr = 0; rr < 2; ++rr) {
+    l[rr] += __shfl_xor_sync(0xffffffffu, l[rr], 1);
+    l[rr] += __shfl_xor_sync(0xffffffffu, l[rr], 2);
+    const int row = g + 8 * rr;
+    if (row >= S * S) continue;
+    const int y = wi * S + row / S, x = wj * S + row % S;
+    const bool qv = y < a.g.Hv && x < a.g.Wv;
+    const float inv = (qv && l[rr] > 0.f) ? 1.f / l[rr] : 0.f;
+    const long long tok = (static_cast<long long>(f) * a.g.Hp + y) * a.g.Wp + x;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+      *reinterpret_cast<uint32_t*>(oh + tok * D + 8 * nt + 2 * t) =
+          pack_bf16(o[nt][2 * rr] * inv, o[nt][2 * rr + 1] * inv);
+  }
+}
+
+// fp32: one thread per query token
+template <int S>
+__global__ void __launch_bounds__(128) sel_kernel_f32(const SelArgs a) {
+  const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long per_head = static_cast<long long>(a.F) * a.g.Hp * a.g.Wp;
+  if (tid >= per_head * a.H) return;
+  const int h = static_cast<int>(tid / per_head);
+  const long long n = tid - h * per_head;
+  const int f = static_cast<int>(n / (a.g.Hp * a.g.Wp));
+  const int o2 = static_cast<int>(n - static_cast<long long>(f) * a.g.Hp * a.g.Wp);
+  const int y = o2 / a.g.Wp, x = o2 - y * a.g.Wp;
+  const long long img_hs = per_head * D;
+  const long long spec_hs = static_cast<long long>(a.F) * a.g.ns * D;
+  float* out = reinterpret_cast<float*>(a.o_sel) + h * img_hs + n * D;
+  if (y >= a.g.Hv || x >= a.g.Wv) {
+    for (int d = 0; d < D; ++d) out[d] = 0.f;
+    return;
+  }
+  const int r = f * a.rpf + (y / S) * (a.g.Wp / S) + x / S;
+  const int* idx = a.idx + (static_cast<long long>(h) * a.R + r) * a.topk;
+  for (int j = 0; j < a.topk; ++j)
+    if (idx[j] < 0 || idx[j] >= a.R) {
+      set_error(a.err, ERR_BOUNDS);
+      for (int d = 0; d < D; ++d) out[d] = 0.f;
+      return;
+    }
+  const float* q = reinterpret_cast<const float*>(a.q_img) + h * img_hs + n * D;
+  const float* kh = reinterpret_cast<const float*>(a.k_img) + h * img_hs;
+  const float* vh = reinterpret_cast<const float*>(a.v_img) + h * img_hs;
+  const float* ksh = reinterpret_cast<const float*>(a.k_spec) + h * spec_hs;
+  const float* vsh = reinterpret_cast<const float*>(a.v_spec) + h * spec_hs;
+  float qr[D], acc[D];
+  for (int d = 0; d < D; ++d) { qr[d] = q[d]; acc[d] = 0.f; }
+  const int nk_dyn = a.topk * S * S;
+  const int nkeys = nk_dyn + a.n_fixed * (a.g.ns + a.g.Hp * a.g.Wp);
+  const float scale = a.scale_log2 / LOG2E;
+  float mx = -INFINITY, l = 0.f;
+  for (int p = 0; p < nkeys; ++p) {
+    long long off;
+    bool spec;
+    bool ok;
+    if (p < nk_dyn) {
+      const int2 rb = region_base<S>(a, idx[p / (S * S)]);
+      ok = key_src<S>(a, &rb, p % (S * S), S * S, S * S, off, spec);
+    } else {
+      ok = key_src<S>(a, nullptr, p, nk_dyn, nkeys, off, spec);
+    }
+    if (!ok) continue;
+    const float* kp = (spec ? ksh : kh) + off * D;
+    const float* vp = (spec ? vsh : vh) + off * D;
+    float sc = 0.f;
+    for (int d = 0; d < D; ++d) sc = fmaf(qr[d], kp[d], sc);
+    sc *= scale;
+    const float mn = fmaxf(mx, sc);
+    const float al = expf(mx - mn);
+    const float pw = expf(sc - mn);
+    l = l * al + pw;
+    for (int d = 0; d < D; ++d) acc[d] = acc[d] * al + pw * vp[d];
+    mx = mn;
+  }
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  for (int d = 0; d < D; ++d) out[d] = acc[d] * inv;
+}
+
+template <int S>
+cudaError_t launch_sel_s(const SelArgs& a, bool fp32, cudaStream_t st) {
+  if (fp32) {
+    const long long n = static_cast<long long>(a.H) * a.F * a.g.Hp * a.g.Wp;
+    sel_kernel_f32<S><<<static_cast<unsigned>((n + 127) / 128), 128, 0, st>>>(a);
+  } else {
+    const int sm = SEL_WARPS * SEL_WARP_SMEM;
+    cudaError_t e = cudaFuncSetAttribute(sel_kernel_bf16<S>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    if (e != cudaSuccess) return e;
+    const long long w = static_cast<long long>(a.H) * a.R;
+    sel_kernel_bf16<S><<<static_cast<unsigned>((w + SEL_WARPS - 1) / SEL_WARPS), SEL_WARPS * 32, sm, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_sel(const SelArgs& a, bool fp32, cudaStream_t st) {
+  switch (a.s) {
+    case 1: return launch_sel_s<1>(a, fp32, st);
+    case 2: return launch_sel_s<2>(a, fp32, st);
+    case 4: return launch_sel_s<4>(a, fp32, st);
+    case 8:
+      if (fp32) return launch_sel_s<8>(a, true, st);
+      return cudaErrorInvalidValue;
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace gsa

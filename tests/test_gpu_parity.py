@@ -1,0 +1,164 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the CPU oracle on
+the same seeded inputs (see gpu_helpers for the acceptance bars)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gsa_inputs import CONFIGS, GSAConfig, make_inputs, to_f64_numpy
+from gpu_helpers import assert_close, compare_head, run_gpu
+
+pytestmark = pytest.mark.gpu
+
+# small cases that still span several tiles and ragged tails
+RAGGED_BF16 = GSAConfig("ragged_bf16", 3, 12, 12, 12, 12, 2, 2, 64, 4, 8, "bf16")          # R=27
+MULTI_TILE_BF16 = GSAConfig("multi_tile_bf16", 6, 24, 24, 24, 24, 5, 2, 64, 4, 32, "bf16")  # R=216
+S2_BF16 = GSAConfig("s2_bf16", 2, 10, 14, 10, 14, 1, 2, 64, 2, 12, "bf16")                  # R=70
+PAD_VGGT_BF16 = GSAConfig("pad_vggt_bf16", 5, 10, 11, 12, 12, 3, 2, 64, 4, 6, "bf16", (0, 3))
+NO_SPECIAL_BF16 = GSAConfig("no_special_bf16", 4, 16, 16, 16, 16, 0, 1, 64, 4, 5, "bf16")
+PAD_F32 = GSAConfig("pad_vggt_f32", 4, 7, 7, 8, 8, 2, 2, 64, 2, 5, "fp32", (1,))
+
+SMALL = [CONFIGS["tiny_fp32"], RAGGED_BF16, MULTI_TILE_BF16, S2_BF16, PAD_VGGT_BF16,
+         NO_SPECIAL_BF16, PAD_F32]
+
+
+def _cuda_inputs(cfg, seed=0):
+    return {k: v.cuda() for k, v in make_inputs(cfg, seed=seed).items()}
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=[c.name for c in SMALL])
+def test_small_configs_full_parity(cfg):
+    x = _cuda_inputs(cfg)
+    res = run_gpu(cfg, x)
+    for h in range(cfg.num_heads):
+        compare_head(cfg, x, res, h)
+    # the caller's copy of the selection equals the workspace copy
+    assert torch.equal(res["idx"], res["idx_ws"])
+
+
+@pytest.mark.parametrize("cfg", [CONFIGS["tiny_fp32"], PAD_VGGT_BF16], ids=["tiny_fp32", "pad_vggt_bf16"])
+@pytest.mark.parametrize("mode", ["comp_only", "sel_only"])
+def test_gate_modes_isolate_branches(cfg, mode):
+    x = _cuda_inputs(cfg)
+    res = run_gpu(cfg, x, gate_mode=mode)
+    for h in range(cfg.num_heads):
+        compare_head(cfg, x, res, h, gate_mode=mode)
+
+
+@pytest.mark.parametrize("cfg", [CONFIGS["tiny_fp32"], RAGGED_BF16, S2_BF16],
+                         ids=["tiny_fp32", "ragged_bf16", "s2_bf16"])
+def test_selection_with_every_region_equals_dense(cfg):
+    """top-k = number of regions: the selection branch is dense attention over
+    all image tokens (independent of the selection order)."""
+    k = cfg.num_regions
+    if k > 64:
+        k = None
+        cfg = cfg.with_(num_frames=1)
+        k = cfg.num_regions
+    x = _cuda_inputs(cfg)
+    res = run_gpu(cfg, x, gate_mode="sel_only", topk=k)
+    d = cfg.head_dim
+    valid = np.tile(oracle.valid_grid(cfg.grid_h, cfg.grid_w, cfg.pad_h, cfg.pad_w).reshape(-1),
+                    cfg.num_frames)
+    for h in range(cfg.num_heads):
+        q = to_f64_numpy(x["q_img"][h]).reshape(-1, d)
+        kk = to_f64_numpy(x["k_img"][h]).reshape(-1, d)
+        v = to_f64_numpy(x["v_img"][h]).reshape(-1, d)
+        want = oracle.attention(q, kk, v, 1 / np.sqrt(d), valid)
+        got = res["o_img"][h].float().cpu().numpy().reshape(-1, d)
+        assert_close("O_img(all regions)", got[valid], want[valid], cfg)
+        assert sorted(res["idx"][h, 0].tolist()) == list(range(k))
+
+
+def test_pi3_32_frames_parity():
+    cfg = CONFIGS["pi3_f32"]
+    x = _cuda_inputs(cfg)
+    res = run_gpu(cfg, x)
+    tot_checked = tot_under = 0
+    for h in (0, 9, 15):
+        c, u = compare_head(cfg, x, res, h)
+        tot_checked += c
+        tot_under += u
+    assert tot_checked > 0
+
+
+def _sample_windows(cfg, n, seed):
+    rng = np.random.default_rng(seed)
+    R, rpf = cfg.num_regions, cfg.regions_per_frame
+    w = set(rng.choice(R, size=n, replace=False).tolist())
+    w |= {0, R - 1, rpf - 1, R - rpf}          # first/last, frame edges (ragged pad regions)
+    for f in cfg.fixed_frames:
+        w.add(f * rpf + rpf // 2)               # windows inside fixed-context frames
+    return np.array(sorted(w))
+
+
+@pytest.mark.parametrize("name", ["pi3_f128", "vggt_f256", "pi3_f1000"])
+def test_full_size_sampled_parity(name):
+    """Full-size workloads in the benchmark's launch configuration; the oracle
+    checks a seeded sample of windows and special rows of two heads."""
+    cfg = CONFIGS[name]
+    x = make_inputs(cfg, seed=0, device="cuda")
+    res = run_gpu(cfg, x)
+    for h in (0, cfg.num_heads - 1):
+        win = _sample_windows(cfg, 40, seed=h)
+        srows = np.random.default_rng(100 + h).choice(cfg.num_spec, size=12, replace=False)
+        compare_head(cfg, x, res, h, windows=win, spec_rows=np.sort(srows))
+    # every selected region index of every head is a valid candidate
+    idx = res["idx"]
+    assert int(idx.min()) >= 0 and int(idx.max()) < cfg.num_regions
+    srt = torch.sort(idx, dim=-1).values
+    assert bool((srt[..., 1:] != srt[..., :-1]).all())
+
+
+@pytest.mark.parametrize("cfg", [CONFIGS["tiny_fp32"], PAD_VGGT_BF16, RAGGED_BF16],
+                         ids=["tiny_fp32", "pad_vggt_bf16", "ragged_bf16"])
+def test_dense_kernel_parity(cfg):
+    import sparse_global_attention_b200 as gsa
+    x = make_inputs(cfg, seed=3)
+    H, F, ns, Hp, Wp, d = cfg.num_heads, cfg.num_frames, cfg.num_special, cfg.pad_h, cfg.pad_w, 64
+
+    def dense_layout(spec, img):
+        return torch.cat([spec, img.reshape(H, F, Hp * Wp, d)], dim=2).reshape(H, -1, d).contiguous()
+
+    q = dense_layout(x["q_spec"], x["q_img"]).cuda()
+    k = dense_layout(x["k_spec"], x["k_img"]).cuda()
+    v = dense_layout(x["v_spec"], x["v_img"]).cuda()
+    layer = gsa.GSALayer.from_workload(cfg)
+    o = layer.dense(q, k, v)
+    torch.cuda.synchronize()
+    layer.close()
+    valid = oracle.dense_token_layout_valid(F, ns, cfg.grid_h, cfg.grid_w, Hp, Wp)
+    for h in range(H):
+        want = oracle.dense_attention(to_f64_numpy(q[h]), to_f64_numpy(k[h]), to_f64_numpy(v[h]), valid)
+        got = o[h].float().cpu().numpy()
+        assert_close("dense", got[valid], want[valid], cfg)
+        assert np.all(got[~valid] == 0)
+
+
+def test_dense_kernel_sampled_pi3_32():
+    import sparse_global_attention_b200 as gsa
+    cfg = CONFIGS["pi3_f32"]
+    x = make_inputs(cfg, seed=1, device="cuda")
+    H, F, d = cfg.num_heads, cfg.num_frames, 64
+
+    def dense_layout(spec, img):
+        return torch.cat([spec, img.reshape(H, F, -1, d)], dim=2).reshape(H, -1, d).contiguous()
+
+    q, k, v = (dense_layout(x[n + "_spec"], x[n + "_img"]) for n in "qkv")
+    layer = gsa.GSALayer.from_workload(cfg)
+    o = layer.dense(q, k, v)
+    torch.cuda.synchronize()
+    layer.close()
+    rows = np.sort(np.random.default_rng(0).choice(q.shape[1], size=64, replace=False))
+    for h in (0, 15):
+        want = oracle.dense_attention(to_f64_numpy(q[h]), to_f64_numpy(k[h]), to_f64_numpy(v[h]), rows=rows)
+        assert_close("dense", o[h].float().cpu().numpy()[rows], want, cfg)
+
+
+def test_repeated_forward_is_deterministic():
+    cfg = MULTI_TILE_BF16
+    x = _cuda_inputs(cfg)
+    a = run_gpu(cfg, x)
+    b = run_gpu(cfg, x)
+    assert torch.equal(a["o_img"], b["o_img"]) and torch.equal(a["idx"], b["idx"])
+    assert torch.equal(a["o_spec"], b["o_spec"])
