@@ -154,6 +154,39 @@ GSA_API const char *gsa_strerror(int code);
 /* Free the workspace and the context; NULL is accepted. */
 GSA_API void gsa_destroy(gsa_ctx *ctx);
 
+/* ---- allocation-free variant -------------------------------------------------
+ * The notes describe no counterpart of this entry point; it serves callers that
+ * cannot call cudaMalloc: a host program or serving engine that reserves all
+ * device memory up front and hands the layer only its inputs and outputs, or a
+ * latency-critical loop where an allocation's implicit synchronisation is not
+ * acceptable.
+ *
+ * gsa_special_attention_noalloc computes the special-token output of
+ * gsa_forward (every special token attends to every special token and every
+ * valid image token, scale softmax_scale or 1/sqrt(64) when 0) for bf16
+ * tensors with the layouts of gsa_forward:
+ *   q_spec, k_spec, v_spec, o_spec : [H][F][num_special][64]
+ *   k_img, v_img                   : [H][F][pad_h][pad_w][64]
+ * It creates no context and allocates no memory: the per-split partial results
+ * live in one static device array of GSA_NOALLOC_SCRATCH_BYTES per GPU, held
+ * by every GPU that loads the library until the process exits.
+ *   - The first call on a device, with that device current, looks up the
+ *     array's device address (cudaGetSymbolAddress) and caches it; make that
+ *     first call before any stream capture.
+ *   - All calls share the array and find the previous call's contents there;
+ *     calls that overlap on the GPU race, so issue them on one stream (or
+ *     otherwise serialise them).
+ *   - Returns GSA_ERR_UNSUPPORTED, without launching anything, when the
+ *     partials (n_split * H * F * num_special * 264 bytes, n_split chosen as in
+ *     gsa_forward) would exceed the array; GSA_ERR_INVALID_ARG for NULL
+ *     pointers or bad sizes; GSA_ERR_CUDA if a launch fails. */
+#define GSA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+GSA_API int gsa_special_attention_noalloc(const void *q_spec, const void *k_spec, const void *v_spec,
+                                          const void *k_img, const void *v_img, void *o_spec,
+                                          int num_heads, int num_frames, int num_special,
+                                          int grid_h, int grid_w, int pad_h, int pad_w,
+                                          float softmax_scale, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -21,7 +21,7 @@ GSA_GATE_LEARNED, GSA_GATE_COMP_ONLY, GSA_GATE_SEL_ONLY = 0, 1, 2
 GATE_MODES = {"learned": 0, "comp_only": 1, "sel_only": 2}
 EXPORTED = ("gsa_create", "gsa_workspace_bytes", "gsa_forward", "gsa_dense_forward",
             "gsa_get_intermediate", "gsa_set_profiling", "gsa_get_kernel_times",
-            "gsa_get_status", "gsa_strerror", "gsa_destroy")
+            "gsa_get_status", "gsa_strerror", "gsa_destroy", "gsa_special_attention_noalloc")
 
 
 class gsa_config(ctypes.Structure):
@@ -166,6 +166,21 @@ def gsa_strerror(code: int) -> str:
 def gsa_destroy(ctx):
     if ctx:
         load_library().gsa_destroy(ctx)
+
+
+def gsa_special_attention_noalloc(q_spec, k_spec, v_spec, k_img, v_img, o_spec, num_heads,
+                                  num_frames, num_special, grid_h, grid_w, pad_h, pad_w,
+                                  softmax_scale=0.0, stream=0) -> int:
+    """Special-token attention for callers that cannot allocate device memory
+    (a host that owns all GPU memory, or a loop that cannot pay for an
+    allocation's synchronisation): no context, partials in the library's static
+    device array.  Pointers as ints; returns the C status code."""
+    lib = load_library()
+    fn = lib.gsa_special_attention_noalloc
+    fn.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_int] * 7 + [ctypes.c_float, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    return fn(q_spec, k_spec, v_spec, k_img, v_img, o_spec, num_heads, num_frames, num_special,
+              grid_h, grid_w, pad_h, pad_w, float(softmax_scale), stream or None)
 
 
 # ---- torch convenience wrapper (marshalling only) ------------------------------------
