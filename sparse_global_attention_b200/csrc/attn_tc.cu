@@ -96,6 +96,44 @@ __device__ __noinline__ uint32_t chunk_valid(int km, Grid g, int nk, long long k
   return m;
 }
 
+// c ? a : b through an explicit selp, so that chains of these over a
+// register array stay register selects (never an indexed local-memory load)
+__device__ __forceinline__ uint32_t sel_if(bool c, uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("{\n .reg .pred p;\n setp.ne.u32 p, %3, 0;\n selp.b32 %0, %1, %2, p;\n}\n"
+      : "=r"(r)
+      : "r"(a), "r"(b), "r"(static_cast<uint32_t>(c)));
+  return r;
+}
+
+// v[e] for a runtime e in [0, 32): five levels of selects on the bits of e
+__device__ __forceinline__ uint32_t pick32(const uint32_t* v, int e) {
+  uint32_t t[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) t[i] = sel_if(e & 16, v[i + 16], v[i]);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) t[i] = sel_if(e & 8, t[i + 8], t[i]);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) t[i] = sel_if(e & 4, t[i + 4], t[i]);
+#pragma unroll
+  for (int i = 0; i < 2; ++i) t[i] = sel_if(e & 2, t[i + 2], t[i]);
+  return sel_if(e & 1, t[1], t[0]);
+}
+
+// max of 32 values with 4 independent chains
+__device__ __forceinline__ float max32(const uint32_t* v) {
+  float m0 = __uint_as_float(v[0]), m1 = __uint_as_float(v[1]), m2 = __uint_as_float(v[2]),
+        m3 = __uint_as_float(v[3]);
+#pragma unroll
+  for (int e = 4; e < 32; e += 4) {
+    m0 = fmaxf(m0, __uint_as_float(v[e]));
+    m1 = fmaxf(m1, __uint_as_float(v[e + 1]));
+    m2 = fmaxf(m2, __uint_as_float(v[e + 2]));
+    m3 = fmaxf(m3, __uint_as_float(v[e + 3]));
+  }
+  return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+}
+
 __device__ __forceinline__ void apply_mask(uint32_t* v, uint32_t msk) {
 #pragma unroll
   for (int e = 0; e < 32; ++e) v[e] = ((msk >> e) & 1u) ? v[e] : 0xff800000u;   // -inf
@@ -321,7 +359,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // key validity of the tile's four 32-key chunks (all ones unless ragged or padded)
       uint32_t vm[4] = {~0u, ~0u, ~0u, ~0u};
       if (km != MASK_NONE || kb + TBN > nk) {
-#pragma unroll 1
+#pragma unroll
         for (int c = 0; c < 4; ++c) vm[c] = chunk_valid(km, a.g, nk, kb + 32 * c);
       }
       float mx = -INFINITY;
@@ -331,12 +369,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tmem_ld64(tS, v);
         tmem_ld64(tS + 64, v + 64);
         tmem_wait_ld();
+        float cm[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           if (vm[c] != ~0u) apply_mask(v + 32 * c, vm[c]);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(v[32 * c + e]));
+          cm[c] = max32(v + 32 * c);
         }
+        mx = fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3]));
         rescale(mx, m, l, j, qi, tO, bars, a.err, ok, sl2);
         if (!ok) break;
         const float mb = (m == -INFINITY) ? 0.f : m * sl2;
@@ -364,32 +403,32 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tmem_wait_ld();
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
-            const uint32_t msk = vm[2 * hf + c];
+            const uint32_t msk = sel_if(hf, vm[2 + c], vm[c]);
             if (msk != ~0u) apply_mask(v + 32 * c, msk);
+            const float cmax = max32(v + 32 * c);
+            mx = fmaxf(mx, cmax);
             uint32_t cb = 0;
+            if (cmax > thr) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const float x = __uint_as_float(v[32 * c + e]);
-              mx = fmaxf(mx, x);
-              cb |= (x > thr ? 1u : 0u) << e;
+              for (int e = 0; e < 32; ++e) cb |= (__uint_as_float(v[32 * c + e]) > thr ? 1u : 0u) << e;
             }
             // rare: a score beats the current k-th; take the candidates in column order
             while (cb) {
               const int e = __ffs(cb) - 1;
               cb &= cb - 1;
-              float x = __uint_as_float(v[32 * c]);
-#pragma unroll
-              for (int q = 1; q < 32; ++q)
-                if (q == e) x = __uint_as_float(v[32 * c + q]);
+              const float x = __uint_as_float(pick32(v + 32 * c, e));
               if (!(x > thr)) continue;
               const int col = static_cast<int>(kb) + 64 * hf + 32 * c + e;
               if (a.n_fixed && is_fixed_region(a, col)) continue;
               topk_insert<KC>(ts, ti, x, col);
-              float t = ts[KC - 1];
+              if (a.kc == KC) {
+                thr = ts[KC - 1];
+              } else {
+                uint32_t t = __float_as_uint(ts[KC - 1]);
 #pragma unroll
-              for (int p = 0; p < KC; ++p)
-                if (p == a.kc - 1) t = ts[p];
-              thr = t;
+                for (int p = 0; p < KC; ++p) t = sel_if(p == a.kc - 1, __float_as_uint(ts[p]), t);
+                thr = __uint_as_float(t);
+              }
             }
           }
         }
@@ -403,8 +442,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           uint32_t v[64];
           tmem_ld64(tS + 64 * hf, v);
           tmem_wait_ld();
-          if (vm[2 * hf] != ~0u) apply_mask(v, vm[2 * hf]);
-          if (vm[2 * hf + 1] != ~0u) apply_mask(v + 32, vm[2 * hf + 1]);
+          const uint32_t m0 = sel_if(hf, vm[2], vm[0]), m1 = sel_if(hf, vm[3], vm[1]);
+          if (m0 != ~0u) apply_mask(v, m0);
+          if (m1 != ~0u) apply_mask(v + 32, m1);
           uint32_t pk[32];
 #pragma unroll
           for (int e = 0; e < 64; e += 2) {
