@@ -45,7 +45,6 @@ using namespace tc;
 constexpr int TBM = 128;                 // rows per query tile
 constexpr int TBN = 128;                 // keys per tile
 constexpr int TILE = TBN * 128;          // bytes of one 128x64 bf16 tile
-constexpr int NST = 3;                   // K/V ring depth
 constexpr int NTHREADS = 320;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float RESCALE_LOG2 = 8.f;      // rescale O when the max grows by > 2^8
@@ -56,27 +55,40 @@ constexpr uint32_t IDESC_PV = idesc_bf16(128, 64, true);
 template <int KC>
 struct Lay {
   static constexpr bool TOPK = KC > 0;
+  static constexpr int NST = TOPK ? 2 : 3;             // K/V ring depth
   static constexpr int QT = TOPK ? 2 : 1;              // tiles per query tile (hi[, lo])
   static constexpr int KT = TOPK ? 3 : 2;              // tiles per stage: K hi, [K lo], V
   static constexpr int KV = 2 * QT * TILE;             // Q_i hi at i*TILE, lo at (2+i)*TILE
   static constexpr int STAGE = KT * TILE;
-  static constexpr int BAR = KV + NST * STAGE;
-  // barriers: q_full, full[NST], empty[NST], s_full[2], p_full[2], pv_done[2], fin
-  static constexpr int NBAR = 1 + 2 * NST + 6 + 1;
+  static constexpr int P = KV + NST * STAGE;           // P_i (bf16, 128 x 128) at P + i * 2 * TILE
+  static constexpr int BAR = P + 4 * TILE;
+  // barriers: q_full, full[NST], empty[NST], s_full[2], s_free[2], p_full[2], pv_done[2], fin
+  static constexpr int NBAR = 1 + 2 * NST + 8 + 1;
   static constexpr int TMEM_SLOT = BAR + NBAR * 8;
   static constexpr int BYTES = TMEM_SLOT + 16 + 1024;   // + alignment slack
 };
 
 struct Bars {
   uint32_t base;
+  int nst;
   __device__ uint32_t q_full() const { return base; }
   __device__ uint32_t full(int s) const { return base + 8 * (1 + s); }
-  __device__ uint32_t empty(int s) const { return base + 8 * (1 + NST + s); }
-  __device__ uint32_t s_full(int i) const { return base + 8 * (1 + 2 * NST + i); }
-  __device__ uint32_t p_full(int i) const { return base + 8 * (3 + 2 * NST + i); }
-  __device__ uint32_t pv_done(int i) const { return base + 8 * (5 + 2 * NST + i); }
-  __device__ uint32_t fin() const { return base + 8 * (7 + 2 * NST); }
+  __device__ uint32_t empty(int s) const { return base + 8 * (1 + nst + s); }
+  __device__ uint32_t s_full(int i) const { return base + 8 * (1 + 2 * nst + i); }
+  __device__ uint32_t s_free(int i) const { return base + 8 * (3 + 2 * nst + i); }
+  __device__ uint32_t p_full(int i) const { return base + 8 * (5 + 2 * nst + i); }
+  __device__ uint32_t pv_done(int i) const { return base + 8 * (7 + 2 * nst + i); }
+  __device__ uint32_t fin() const { return base + 8 * (9 + 2 * nst); }
 };
+
+// Stores 8 bf16 (16 bytes) of row r, keys [8*c16, 8*c16+8), into a 128 x 128
+// K-major tile with 128-byte swizzle: two 64-key atoms of 16 KB.
+__device__ __forceinline__ void st_p16(uint32_t pbase, int r, int c16, uint4 v) {
+  const uint32_t addr = pbase + (c16 >> 3) * 16384 + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
 
 __device__ __forceinline__ int tile_seg(const AttnArgs& a, int tt, long long& kb) {
   const int seg = (a.nseg > 1 && tt >= a.tiles0) ? 1 : 0;
@@ -214,7 +226,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   uint8_t* sgen = smem_raw + (sbase - raw);
-  const Bars bars{sbase + L::BAR};
+  const Bars bars{sbase + L::BAR, L::NST};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sgen + L::TMEM_SLOT);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -226,12 +238,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bars.q_full(), 1);
-    for (int s = 0; s < NST; ++s) {
+    for (int s = 0; s < L::NST; ++s) {
       mbar_init(bars.full(s), 1);
       mbar_init(bars.empty(s), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bars.s_full(i), 1);
+      mbar_init(bars.s_free(i), TBM);
       mbar_init(bars.p_full(i), TBM);
       mbar_init(bars.pv_done(i), 1);
     }
@@ -246,88 +259,112 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && ntile > 0) {
-      prefetch_tmap(&tm_q);
-      prefetch_tmap(&tm_k0);
-      prefetch_tmap(&tm_v0);
+    if (ntile > 0) {
+      const bool leader = elect_one();
       const int qy = h * a.n_q + row0;
-      mbar_expect_tx(bars.q_full(), 2 * L::QT * TILE);
-      tma_load_2d(sbase + 0 * TILE, &tm_q, 0, qy, bars.q_full());
-      tma_load_2d(sbase + 1 * TILE, &tm_q, 0, qy + TBM, bars.q_full());
-      if constexpr (L::TOPK) {
-        tma_load_2d(sbase + 2 * TILE, &tm_qlo, 0, qy, bars.q_full());
-        tma_load_2d(sbase + 3 * TILE, &tm_qlo, 0, qy + TBM, bars.q_full());
+      if (leader) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k0);
+        prefetch_tmap(&tm_v0);
+        mbar_expect_tx(bars.q_full(), 2 * L::QT * TILE);
+        tma_load_2d(sbase + 0 * TILE, &tm_q, 0, qy, bars.q_full());
+        tma_load_2d(sbase + 1 * TILE, &tm_q, 0, qy + TBM, bars.q_full());
+        if constexpr (L::TOPK) {
+          tma_load_2d(sbase + 2 * TILE, &tm_qlo, 0, qy, bars.q_full());
+          tma_load_2d(sbase + 3 * TILE, &tm_qlo, 0, qy + TBM, bars.q_full());
+        }
       }
+      __syncwarp();
       int issued = 0;
       for (int it = 0; it < ntile; ++it) {
-        const int s = it % NST;
-        if (it >= NST && !mbar_wait(bars.empty(s), ((it / NST) - 1) & 1, a.err)) break;
+        const int s = it % L::NST;
+        if (it >= L::NST &&
+            !__all_sync(0xffffffffu, mbar_wait(bars.empty(s), ((it / L::NST) - 1) & 1, a.err)))
+          break;
         long long kb;
         const int seg = tile_seg(a, t_begin + it, kb);
         const int y = static_cast<int>(static_cast<long long>(h) * a.n_k[seg] + kb);
         const uint32_t st = sbase + L::KV + s * L::STAGE;
-        mbar_expect_tx(bars.full(s), L::KT * TILE);
-        tma_load_2d(st, seg ? &tm_k1 : &tm_k0, 0, y, bars.full(s));
-        if constexpr (L::TOPK) tma_load_2d(st + TILE, &tm_klo, 0, y, bars.full(s));
-        tma_load_2d(st + (L::KT - 1) * TILE, seg ? &tm_v1 : &tm_v0, 0, y, bars.full(s));
+        if (leader) {
+          mbar_expect_tx(bars.full(s), L::KT * TILE);
+          tma_load_2d(st, seg ? &tm_k1 : &tm_k0, 0, y, bars.full(s));
+          if constexpr (L::TOPK) tma_load_2d(st + TILE, &tm_klo, 0, y, bars.full(s));
+          tma_load_2d(st + (L::KT - 1) * TILE, seg ? &tm_v1 : &tm_v0, 0, y, bars.full(s));
+        }
+        __syncwarp();
         ++issued;
       }
       // drain: every issued copy has landed before the CTA may exit
-      for (int it = max(0, issued - NST); it < issued; ++it)
-        mbar_wait(bars.full(it % NST), (it / NST) & 1, a.err);
+      for (int it = max(0, issued - L::NST); it < issued; ++it)
+        mbar_wait(bars.full(it % L::NST), (it / L::NST) & 1, a.err);
       mbar_wait(bars.q_full(), 0, a.err);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && ntile > 0) {
-      bool ok = mbar_wait(bars.q_full(), 0, a.err);
+    // The whole warp runs the loop (operands stay warp-uniform); one elected
+    // lane issues every MMA and commit.  Descriptors are built once and
+    // advanced by adding to their start-address field (16-byte units).
+    if (ntile > 0) {
+      const bool leader = elect_one();
+      const uint64_t dq0 = sdesc_sw128(sbase, 16, 1024);                    // Q_0 hi
+      const uint64_t dk0 = sdesc_sw128(sbase + L::KV, 16, 1024);            // stage 0 K hi
+      const uint64_t dv0 = sdesc_sw128(sbase + L::KV + (L::KT - 1) * TILE, 8192, 1024);   // stage 0 V
+      const uint64_t dp0 = sdesc_sw128(sbase + L::P, 16, 1024);             // P_0
+      constexpr uint32_t T16 = TILE >> 4, ST16 = L::STAGE >> 4;
+      bool ok = __all_sync(0xffffffffu, mbar_wait(bars.q_full(), 0, a.err));
       tc_fence_after();
       for (int j = 0; ok && j <= ntile; ++j) {
         if (j < ntile) {
-          ok = mbar_wait(bars.full(j % NST), (j / NST) & 1, a.err);
+          ok = __all_sync(0xffffffffu, mbar_wait(bars.full(j % L::NST), (j / L::NST) & 1, a.err));
           if (!ok) break;
           tc_fence_after();
+          // S_{i,j} = Q_i K_j^T (guide: + Q_i^hi K_j^lo + Q_i^lo K_j^hi), as soon as
+          // the softmax warps have read S_{i,j-1} into registers
+          const uint64_t dk = dk0 + (j % L::NST) * ST16;
+          for (int i = 0; i < 2 && ok; ++i) {
+            if (j > 0) {
+              ok = __all_sync(0xffffffffu, mbar_wait(bars.s_free(i), (j - 1) & 1, a.err));
+              if (!ok) break;
+              tc_fence_after();
+            }
+            const uint64_t dq = dq0 + i * T16;
+            if (leader) {
+#pragma unroll
+              for (int ks = 0; ks < 4; ++ks) {
+                mma_bf16_ss(tmem + 128 * i, dq + 2 * ks, dk + 2 * ks, IDESC_QK, ks > 0 ? 1u : 0u);
+                if constexpr (L::TOPK) {
+                  mma_bf16_ss(tmem + 128 * i, dq + 2 * ks, dk + T16 + 2 * ks, IDESC_QK, 1u);
+                  mma_bf16_ss(tmem + 128 * i, dq + 2 * T16 + 2 * ks, dk + 2 * ks, IDESC_QK, 1u);
+                }
+              }
+              mma_commit(bars.s_full(i));
+            }
+            __syncwarp();
+          }
         }
-        for (int i = 0; i < 2 && ok; ++i) {
-          if (j > 0) {
-            // O_i += P_{i,j-1} V_{j-1}
-            ok = mbar_wait(bars.p_full(i), (j - 1) & 1, a.err);
+        if (j > 0) {
+          // O_i += P_{i,j-1} V_{j-1}: P from shared memory (K-major), V MN-major
+          const uint64_t dv = dv0 + ((j - 1) % L::NST) * ST16;
+          for (int i = 0; i < 2 && ok; ++i) {
+            ok = __all_sync(0xffffffffu, mbar_wait(bars.p_full(i), (j - 1) & 1, a.err));
             if (!ok) break;
             tc_fence_after();
-            const uint32_t vs = sbase + L::KV + ((j - 1) % NST) * L::STAGE + (L::KT - 1) * TILE;
+            const uint64_t dp = dp0 + i * 2 * T16;
+            if (leader) {
 #pragma unroll
-            for (int ks = 0; ks < TBN / 16; ++ks) {
-              const uint64_t bd = sdesc_sw128(vs + ks * 2048, 8192, 1024);
-              asm volatile(
-                  "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], "
-                  "[%1], %2, %3, p;\n}\n" ::"r"(tmem + 256 + 64 * i),
-                  "r"(tmem + 128 * i + 8 * ks), "l"(bd), "r"(IDESC_PV), "r"((j > 1 || ks > 0) ? 1u : 0u)
-                  : "memory");
+              for (int ks = 0; ks < TBN / 16; ++ks)
+                mma_bf16_ss(tmem + 256 + 64 * i, dp + (ks >> 2) * T16 + (ks & 3) * 2, dv + ks * 128, IDESC_PV,
+                            (j > 1 || ks > 0) ? 1u : 0u);
+              mma_commit(bars.pv_done(i));
             }
-            mma_commit(bars.pv_done(i));
+            __syncwarp();
           }
-          if (j < ntile) {
-            // S_{i,j} = Q_i K_j^T (guide: + Q_i^hi K_j^lo + Q_i^lo K_j^hi)
-            const uint32_t ks0 = sbase + L::KV + (j % NST) * L::STAGE;
-            const uint32_t qs = sbase + i * TILE;
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              const uint64_t ad = sdesc_sw128(qs + 32 * ks, 16, 1024);
-              const uint64_t bd = sdesc_sw128(ks0 + 32 * ks, 16, 1024);
-              mma_bf16_ss(tmem + 128 * i, ad, bd, IDESC_QK, ks > 0 ? 1u : 0u);
-              if constexpr (L::TOPK) {
-                const uint64_t bl = sdesc_sw128(ks0 + TILE + 32 * ks, 16, 1024);
-                const uint64_t al = sdesc_sw128(qs + 2 * TILE + 32 * ks, 16, 1024);
-                mma_bf16_ss(tmem + 128 * i, ad, bl, IDESC_QK, 1u);
-                mma_bf16_ss(tmem + 128 * i, al, bd, IDESC_QK, 1u);
-              }
-            }
-            mma_commit(bars.s_full(i));
-          }
+          if (ok && leader) mma_commit(bars.empty((j - 1) % L::NST));
+          __syncwarp();
         }
-        if (ok && j > 0) mma_commit(bars.empty((j - 1) % NST));
       }
-      mma_commit(bars.fin());
+      if (leader) mma_commit(bars.fin());
+      __syncwarp();
       mbar_wait(bars.fin(), 0, a.err);
     }
   } else {
@@ -338,6 +375,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_off + 128 * qi;
     const uint32_t tO = tmem + lane_off + 256 + 64 * qi;
+    const uint32_t sP = sbase + L::P + qi * 2 * TILE;
     const float sl2 = a.scale_log2;
     float m = -INFINITY, l = 0.f;
     float ts[KC > 0 ? KC : 1], thr = -INFINITY;
@@ -364,11 +402,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       float mx = -INFINITY;
       if constexpr (!L::TOPK) {
-        // whole row of S in registers: one TMEM wait per tile
+        // whole row of S in registers: one TMEM wait per tile, and S_i is handed
+        // back to the MMA warp at once so S_{i,j+1} overlaps this tile's softmax
         uint32_t v[128];
         tmem_ld64(tS, v);
         tmem_ld64(tS + 64, v + 64);
         tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bars.s_free(qi));
         float cm[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -378,6 +419,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mx = fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3]));
         rescale(mx, m, l, j, qi, tO, bars, a.err, ok, sl2);
         if (!ok) break;
+        // P_i is free once PV of the previous tile has completed
+        if (j > 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bars.pv_done(qi), (j - 1) & 1, a.err));
+          if (!ok) break;
+        }
         const float mb = (m == -INFINITY) ? 0.f : m * sl2;
         float l0 = 0.f, l1 = 0.f;
 #pragma unroll
@@ -391,7 +437,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             l1 += p1;
             pk[e >> 1] = pack_bf16(p0, p1);
           }
-          tmem_st16(tS + 16 * c, pk);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            st_p16(sP, r, 4 * c + q, make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]));
         }
         l += l0 + l1;
       } else {
@@ -434,7 +482,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         rescale(mx, m, l, j, qi, tO, bars, a.err, ok, sl2);
         if (!ok) break;
-        // pass 2: P = exp2((S - m) * scale * log2e) as bf16 pairs over S's first 64 columns
+        // pass 2: P = exp2((S - m) * scale * log2e) in bf16 to shared memory; S_i
+        // goes back to the MMA warp after its last half is read
+        if (j > 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bars.pv_done(qi), (j - 1) & 1, a.err));
+          if (!ok) break;
+        }
         const float mb = (m == -INFINITY) ? 0.f : m * sl2;
         float l0 = 0.f, l1 = 0.f;
 #pragma unroll 1
@@ -442,6 +495,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           uint32_t v[64];
           tmem_ld64(tS + 64 * hf, v);
           tmem_wait_ld();
+          if (hf == 1) {
+            tc_fence_before();
+            mbar_arrive(bars.s_free(qi));
+          }
           const uint32_t m0 = sel_if(hf, vm[2], vm[0]), m1 = sel_if(hf, vm[3], vm[1]);
           if (m0 != ~0u) apply_mask(v, m0);
           if (m1 != ~0u) apply_mask(v + 32, m1);
@@ -454,12 +511,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             l1 += p1;
             pk[e >> 1] = pack_bf16(p0, p1);
           }
-          tmem_st32(tS + 32 * hf, pk);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            st_p16(sP, r, 8 * hf + q, make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]));
         }
         l += l0 + l1;
       }
-      tmem_wait_st();
-      tc_fence_before();
+      tc_fence_before();       // O rescale (TMEM stores) before the MMA warp resumes
+      fence_async_smem();      // P stores visible to the tensor cores
       mbar_arrive(bars.p_full(qi));
     }
     // ---- epilogue: O_i row from TMEM ----------------------------------------
