@@ -62,8 +62,9 @@ struct Lay {
   static constexpr int STAGE = KT * TILE;
   static constexpr int P = KV + NST * STAGE;           // P_i (bf16, 128 x 128) at P + i * 2 * TILE
   static constexpr int BAR = P + 4 * TILE;
-  // barriers: q_full, full[NST], empty[NST], s_full[2], s_free[2], p_full[2], pv_done[2], fin
-  static constexpr int NBAR = 1 + 2 * NST + 8 + 1;
+  // barriers: q_full, full[NST], empty[NST], s_full[2], s_free[2], p_full[2], pv_done[2], fin,
+  // turn[2]
+  static constexpr int NBAR = 1 + 2 * NST + 8 + 1 + 2;
   static constexpr int TMEM_SLOT = BAR + NBAR * 8;
   static constexpr int BYTES = TMEM_SLOT + 16 + 1024;   // + alignment slack
 };
@@ -79,7 +80,24 @@ struct Bars {
   __device__ uint32_t p_full(int i) const { return base + 8 * (5 + 2 * nst + i); }
   __device__ uint32_t pv_done(int i) const { return base + 8 * (7 + 2 * nst + i); }
   __device__ uint32_t fin() const { return base + 8 * (9 + 2 * nst); }
+  __device__ uint32_t turn(int i) const { return base + 8 * (10 + 2 * nst + i); }
 };
+
+// one arrival per warp, after every lane's preceding work (fences included)
+__device__ __forceinline__ void warp_arrive(uint32_t bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
+// The two softmax warpgroups take turns on their exponential phase (the MUFU
+// work of a tile): warpgroup 0 runs tile j after warpgroup 1 finished tile
+// j-1, warpgroup 1 runs tile j after warpgroup 0 finished tile j, so one
+// group's exponentials overlap the other's loads, maxima and waits.
+__device__ __forceinline__ bool exp_turn_wait(const Bars& bars, int qi, int j, int* err) {
+  if (qi == 0 && j == 0) return true;
+  const uint32_t par = static_cast<uint32_t>(qi == 0 ? (j - 1) : j) & 1u;
+  return __all_sync(0xffffffffu, mbar_wait(bars.turn(qi), par, err));
+}
 
 // Stores 8 bf16 (16 bytes) of row r, keys [8*c16, 8*c16+8), into a 128 x 128
 // K-major tile with 128-byte swizzle: two 64-key atoms of 16 KB.
@@ -244,9 +262,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bars.s_full(i), 1);
-      mbar_init(bars.s_free(i), TBM);
-      mbar_init(bars.p_full(i), TBM);
+      mbar_init(bars.s_free(i), TBM / 32);     // one arrival per softmax warp
+      mbar_init(bars.p_full(i), TBM / 32);
       mbar_init(bars.pv_done(i), 1);
+      mbar_init(bars.turn(i), TBM / 32);
     }
     mbar_init(bars.fin(), 1);
     fence_mbar_init();
@@ -318,10 +337,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           ok = __all_sync(0xffffffffu, mbar_wait(bars.full(j % L::NST), (j / L::NST) & 1, a.err));
           if (!ok) break;
           tc_fence_after();
-          // S_{i,j} = Q_i K_j^T (guide: + Q_i^hi K_j^lo + Q_i^lo K_j^hi), as soon as
-          // the softmax warps have read S_{i,j-1} into registers
-          const uint64_t dk = dk0 + (j % L::NST) * ST16;
-          for (int i = 0; i < 2 && ok; ++i) {
+        }
+        const uint64_t dk = dk0 + (j % L::NST) * ST16;
+        const uint64_t dv = dv0 + ((j + L::NST - 1) % L::NST) * ST16;
+        for (int i = 0; i < 2 && ok; ++i) {
+          if (j < ntile) {
+            // S_{i,j} = Q_i K_j^T (guide: + Q_i^hi K_j^lo + Q_i^lo K_j^hi), as soon as
+            // warpgroup i has read S_{i,j-1} into registers
             if (j > 0) {
               ok = __all_sync(0xffffffffu, mbar_wait(bars.s_free(i), (j - 1) & 1, a.err));
               if (!ok) break;
@@ -341,11 +363,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             __syncwarp();
           }
-        }
-        if (j > 0) {
-          // O_i += P_{i,j-1} V_{j-1}: P from shared memory (K-major), V MN-major
-          const uint64_t dv = dv0 + ((j - 1) % L::NST) * ST16;
-          for (int i = 0; i < 2 && ok; ++i) {
+          if (j > 0) {
+            // O_i += P_{i,j-1} V_{j-1}: P from shared memory (K-major), V MN-major
             ok = __all_sync(0xffffffffu, mbar_wait(bars.p_full(i), (j - 1) & 1, a.err));
             if (!ok) break;
             tc_fence_after();
@@ -359,9 +378,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             __syncwarp();
           }
-          if (ok && leader) mma_commit(bars.empty((j - 1) % L::NST));
-          __syncwarp();
         }
+        if (ok && j > 0 && leader) mma_commit(bars.empty((j - 1) % L::NST));
+        __syncwarp();
       }
       if (leader) mma_commit(bars.fin());
       __syncwarp();
@@ -409,7 +428,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tmem_ld64(tS + 64, v + 64);
         tmem_wait_ld();
         tc_fence_before();
-        mbar_arrive(bars.s_free(qi));
+        warp_arrive(bars.s_free(qi));
         float cm[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -424,6 +443,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           ok = __all_sync(0xffffffffu, mbar_wait(bars.pv_done(qi), (j - 1) & 1, a.err));
           if (!ok) break;
         }
+        ok = exp_turn_wait(bars, qi, j, a.err);
+        if (!ok) break;
         const float mb = (m == -INFINITY) ? 0.f : m * sl2;
         float l0 = 0.f, l1 = 0.f;
 #pragma unroll
@@ -441,6 +462,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int q = 0; q < 4; ++q)
             st_p16(sP, r, 4 * c + q, make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]));
         }
+        warp_arrive(bars.turn(qi ^ 1));
         l += l0 + l1;
       } else {
         // pass 1, two 64-key halves: row max and the streaming top-k
@@ -488,6 +510,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           ok = __all_sync(0xffffffffu, mbar_wait(bars.pv_done(qi), (j - 1) & 1, a.err));
           if (!ok) break;
         }
+        ok = exp_turn_wait(bars, qi, j, a.err);
+        if (!ok) break;
         const float mb = (m == -INFINITY) ? 0.f : m * sl2;
         float l0 = 0.f, l1 = 0.f;
 #pragma unroll 1
@@ -497,7 +521,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tmem_wait_ld();
           if (hf == 1) {
             tc_fence_before();
-            mbar_arrive(bars.s_free(qi));
+            warp_arrive(bars.s_free(qi));
           }
           const uint32_t m0 = sel_if(hf, vm[2], vm[0]), m1 = sel_if(hf, vm[3], vm[1]);
           if (m0 != ~0u) apply_mask(v, m0);
@@ -515,11 +539,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int q = 0; q < 8; ++q)
             st_p16(sP, r, 8 * hf + q, make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]));
         }
+        warp_arrive(bars.turn(qi ^ 1));
         l += l0 + l1;
       }
       tc_fence_before();       // O rescale (TMEM stores) before the MMA warp resumes
       fence_async_smem();      // P stores visible to the tensor cores
-      mbar_arrive(bars.p_full(qi));
+      warp_arrive(bars.p_full(qi));
     }
     // ---- epilogue: O_i row from TMEM ----------------------------------------
     if (ok && ntile > 0) ok = mbar_wait(bars.pv_done(qi), (ntile - 1) & 1, a.err);
