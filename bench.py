@@ -170,6 +170,23 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def max_over_ranks(v, dist=None, device="cpu"):
+    """Largest value of `v` over all ranks (every rank gets it); the per-step
+    time of a multi-GPU run is the slowest rank's."""
+    if dist is None:
+        return float(v)
+    import torch
+    t = torch.tensor([float(v)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput(world, tokens_per_rank, ms_max):
+    """Whole-job image tokens/s: every rank processes its own workload (weak
+    scaling), the job takes as long as its slowest rank."""
+    return world * tokens_per_rank / (ms_max / 1e3)
+
+
 # ---------------------------------------------------------------------------------------
 # the CPU oracle as the baseline / reference arm
 # ---------------------------------------------------------------------------------------
@@ -269,13 +286,6 @@ def run_b200(args, cfg, rank, world, local, dist):
         if dist is not None:
             dist.barrier()
 
-    def max_over_ranks(v):
-        if dist is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     for _ in range(args.warmup):
         layer.forward(x, out=out)
     torch.cuda.synchronize()
@@ -294,8 +304,8 @@ def run_b200(args, cfg, rank, world, local, dist):
         e1.record(stream)
         torch.cuda.synchronize()
     barrier()
-    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
-    value = world * cfg.num_img_valid / (ms / 1e3)
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dist, dev)
+    value = throughput(world, cfg.num_img_valid, ms)
 
     # ---- per-kernel times (CUDA events recorded by the library on its stream) --
     gsa.gsa_set_profiling(layer.ctx, True)
@@ -402,8 +412,8 @@ def run_b200(args, cfg, rank, world, local, dist):
         f1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        ems = max_over_ranks(f0.elapsed_time(f1) / ke)
-        e2e = {"value": world * cfg.num_img_valid / (ems / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        ems = max_over_ranks(f0.elapsed_time(f1) / ke, dist, dev)
+        e2e = {"value": throughput(world, cfg.num_img_valid, ems), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": round(ems, 3), "steps": ke}
 
     st = layer.status()
