@@ -14,7 +14,8 @@
 //   warp  9    MMA issuer (one thread): S_i = Q_i K^T (SS form, both operands
 //              in 128B-swizzled shared memory) and O_i += P_i V (TS form: P_i
 //              read from TMEM, V as an MN-major shared-memory operand)
-// TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,320), O_1 [320,384).
+// TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,320), O_1 [320,384),
+// P_0 [384,448), P_1 [448,512) (bf16 pairs).
 // Softmax threads read their row of S_i, write P_i (bf16 pairs) back over the
 // first 64 columns of S_i, and rescale O_i in TMEM only when the running max
 // grows by more than 2^8 (lazy rescaling: the stale max keeps every
@@ -55,13 +56,12 @@ constexpr uint32_t IDESC_PV = idesc_bf16(128, 64, true);
 template <int KC>
 struct Lay {
   static constexpr bool TOPK = KC > 0;
-  static constexpr int NST = TOPK ? 2 : 3;             // K/V ring depth
+  static constexpr int NST = 3;                        // K/V ring depth
   static constexpr int QT = TOPK ? 2 : 1;              // tiles per query tile (hi[, lo])
   static constexpr int KT = TOPK ? 3 : 2;              // tiles per stage: K hi, [K lo], V
   static constexpr int KV = 2 * QT * TILE;             // Q_i hi at i*TILE, lo at (2+i)*TILE
   static constexpr int STAGE = KT * TILE;
-  static constexpr int P = KV + NST * STAGE;           // P_i (bf16, 128 x 128) at P + i * 2 * TILE
-  static constexpr int BAR = P + 4 * TILE;
+  static constexpr int BAR = KV + NST * STAGE;
   // barriers: q_full, full[NST], empty[NST], s_full[2], s_free[2], p_full[2], pv_done[2], fin,
   // turn[2]
   static constexpr int NBAR = 1 + 2 * NST + 8 + 1 + 2;
@@ -97,15 +97,6 @@ __device__ __forceinline__ bool exp_turn_wait(const Bars& bars, int qi, int j, i
   if (qi == 0 && j == 0) return true;
   const uint32_t par = static_cast<uint32_t>(qi == 0 ? (j - 1) : j) & 1u;
   return __all_sync(0xffffffffu, mbar_wait(bars.turn(qi), par, err));
-}
-
-// Stores 8 bf16 (16 bytes) of row r, keys [8*c16, 8*c16+8), into a 128 x 128
-// K-major tile with 128-byte swizzle: two 64-key atoms of 16 KB.
-__device__ __forceinline__ void st_p16(uint32_t pbase, int r, int c16, uint4 v) {
-  const uint32_t addr = pbase + (c16 >> 3) * 16384 + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
-               "r"(v.w)
-               : "memory");
 }
 
 __device__ __forceinline__ int tile_seg(const AttnArgs& a, int tt, long long& kb) {
@@ -328,7 +319,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint64_t dq0 = sdesc_sw128(sbase, 16, 1024);                    // Q_0 hi
       const uint64_t dk0 = sdesc_sw128(sbase + L::KV, 16, 1024);            // stage 0 K hi
       const uint64_t dv0 = sdesc_sw128(sbase + L::KV + (L::KT - 1) * TILE, 8192, 1024);   // stage 0 V
-      const uint64_t dp0 = sdesc_sw128(sbase + L::P, 16, 1024);             // P_0
       constexpr uint32_t T16 = TILE >> 4, ST16 = L::STAGE >> 4;
       bool ok = __all_sync(0xffffffffu, mbar_wait(bars.q_full(), 0, a.err));
       tc_fence_after();
@@ -364,15 +354,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             __syncwarp();
           }
           if (j > 0) {
-            // O_i += P_{i,j-1} V_{j-1}: P from shared memory (K-major), V MN-major
+            // O_i += P_{i,j-1} V_{j-1}: P read from TMEM (TS form), V MN-major
             ok = __all_sync(0xffffffffu, mbar_wait(bars.p_full(i), (j - 1) & 1, a.err));
             if (!ok) break;
             tc_fence_after();
-            const uint64_t dp = dp0 + i * 2 * T16;
             if (leader) {
 #pragma unroll
               for (int ks = 0; ks < TBN / 16; ++ks)
-                mma_bf16_ss(tmem + 256 + 64 * i, dp + (ks >> 2) * T16 + (ks & 3) * 2, dv + ks * 128, IDESC_PV,
+                mma_bf16_ts(tmem + 256 + 64 * i, tmem + 384 + 64 * i + 8 * ks, dv + ks * 128, IDESC_PV,
                             (j > 1 || ks > 0) ? 1u : 0u);
               mma_commit(bars.pv_done(i));
             }
@@ -394,7 +383,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_off + 128 * qi;
     const uint32_t tO = tmem + lane_off + 256 + 64 * qi;
-    const uint32_t sP = sbase + L::P + qi * 2 * TILE;
+    const uint32_t tP = tmem + lane_off + 384 + 64 * qi;
     const float sl2 = a.scale_log2;
     float m = -INFINITY, l = 0.f;
     float ts[KC > 0 ? KC : 1], thr = -INFINITY;
@@ -458,9 +447,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             l1 += p1;
             pk[e >> 1] = pack_bf16(p0, p1);
           }
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            st_p16(sP, r, 4 * c + q, make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]));
+          tmem_st16(tP + 16 * c, pk);
         }
         warp_arrive(bars.turn(qi ^ 1));
         l += l0 + l1;
@@ -535,15 +522,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             l1 += p1;
             pk[e >> 1] = pack_bf16(p0, p1);
           }
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            st_p16(sP, r, 8 * hf + q, make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]));
+          tmem_st32(tP + 32 * hf, pk);
         }
         warp_arrive(bars.turn(qi ^ 1));
         l += l0 + l1;
       }
-      tc_fence_before();       // O rescale (TMEM stores) before the MMA warp resumes
-      fence_async_smem();      // P stores visible to the tensor cores
+      tmem_wait_st();          // P (and any O rescale) written to TMEM
+      tc_fence_before();
       warp_arrive(bars.p_full(qi));
     }
     // ---- epilogue: O_i row from TMEM ----------------------------------------
