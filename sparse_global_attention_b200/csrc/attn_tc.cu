@@ -127,11 +127,13 @@ __device__ __forceinline__ uint32_t sel_if(bool c, uint32_t a, uint32_t b) {
   return r;
 }
 
-// v[e] for a runtime e in [0, 32): five levels of selects on the bits of e
-__device__ __forceinline__ uint32_t pick32(const uint32_t* v, int e) {
+// v[e] for a runtime e in [0, 64): the first level folds bits 5 and 4 (four
+// inputs per output, 16 live temporaries), then four levels of selects
+__device__ __forceinline__ uint32_t pick64(const uint32_t* v, int e) {
   uint32_t t[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) t[i] = sel_if(e & 16, v[i + 16], v[i]);
+  for (int i = 0; i < 16; ++i)
+    t[i] = sel_if(e & 32, sel_if(e & 16, v[i + 48], v[i + 32]), sel_if(e & 16, v[i + 16], v[i]));
 #pragma unroll
   for (int i = 0; i < 8; ++i) t[i] = sel_if(e & 8, t[i + 8], t[i]);
 #pragma unroll
@@ -458,34 +460,35 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           uint32_t v[64];
           tmem_ld64(tS + 64 * hf, v);
           tmem_wait_ld();
+          uint32_t cb[2] = {0u, 0u};
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             const uint32_t msk = sel_if(hf, vm[2 + c], vm[c]);
             if (msk != ~0u) apply_mask(v + 32 * c, msk);
             const float cmax = max32(v + 32 * c);
             mx = fmaxf(mx, cmax);
-            uint32_t cb = 0;
             if (cmax > thr) {
 #pragma unroll
-              for (int e = 0; e < 32; ++e) cb |= (__uint_as_float(v[32 * c + e]) > thr ? 1u : 0u) << e;
+              for (int e = 0; e < 32; ++e) cb[c] |= (__uint_as_float(v[32 * c + e]) > thr ? 1u : 0u) << e;
             }
-            // rare: a score beats the current k-th; take the candidates in column order
-            while (cb) {
-              const int e = __ffs(cb) - 1;
-              cb &= cb - 1;
-              const float x = __uint_as_float(pick32(v + 32 * c, e));
-              if (!(x > thr)) continue;
-              const int col = static_cast<int>(kb) + 64 * hf + 32 * c + e;
-              if (a.n_fixed && is_fixed_region(a, col)) continue;
-              topk_insert<KC>(ts, ti, x, col);
-              if (a.kc == KC) {
-                thr = ts[KC - 1];
-              } else {
-                uint32_t t = __float_as_uint(ts[KC - 1]);
+          }
+          // rare: a score beats the current k-th; take the candidates in column
+          // order through one insertion site for the whole half
+          while (cb[0] | cb[1]) {
+            const bool lo = cb[0] != 0;
+            const int e = lo ? __ffs(cb[0]) - 1 : 31 + __ffs(cb[1]);
+            if (lo) cb[0] &= cb[0] - 1; else cb[1] &= cb[1] - 1;
+            const float x = __uint_as_float(pick64(v, e));
+            const int col = static_cast<int>(kb) + 64 * hf + e;
+            if (!(x > thr) || (a.n_fixed && is_fixed_region(a, col))) continue;
+            topk_insert<KC>(ts, ti, x, col);
+            if (a.kc == KC) {
+              thr = ts[KC - 1];
+            } else {
+              uint32_t t = __float_as_uint(ts[KC - 1]);
 #pragma unroll
-                for (int p = 0; p < KC; ++p) t = sel_if(p == a.kc - 1, __float_as_uint(ts[p]), t);
-                thr = __uint_as_float(t);
-              }
+              for (int p = 0; p < KC; ++p) t = sel_if(p == a.kc - 1, __float_as_uint(ts[p]), t);
+              thr = __uint_as_float(t);
             }
           }
         }
@@ -636,6 +639,34 @@ cudaError_t launch_kc(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t s
 }  // namespace
 
 int attn_tc_tiles(long long n) { return static_cast<int>((n + TBN - 1) / TBN); }
+
+void attn_tc_split(int H, long long n_q, int tiles_total, int* tiles_per_split, int* n_split) {
+  // One CTA per SM (TMEM and shared memory), 2 x 128 query rows per CTA.  Take
+  // the fewest key splits that give at least four waves over the 148 SMs, or
+  // more (up to 4x) when that leaves a smaller idle tail in the last wave;
+  // each split keeps at least 16 key tiles.
+  constexpr long long SMS = 148;
+  const long long ctas = static_cast<long long>(H) * ((n_q + 2 * TBM - 1) / (2 * TBM));
+  long long maxs = tiles_total / 16;
+  if (maxs < 1) maxs = 1;
+  if (maxs > 4096) maxs = 4096;
+  long long lo = ctas > 0 ? (4 * SMS + ctas - 1) / ctas : 1;
+  if (lo < 1) lo = 1;
+  if (lo > maxs) lo = maxs;
+  long long best = lo;
+  double best_eff = 0.0;
+  for (long long ns = lo; ns <= maxs && ns <= 4 * lo; ++ns) {
+    const long long tot = ctas * ns;
+    const double eff = static_cast<double>(tot) / static_cast<double>(SMS * ((tot + SMS - 1) / SMS));
+    if (eff > best_eff + 0.02) {
+      best_eff = eff;
+      best = ns;
+    }
+  }
+  const int tps = static_cast<int>((tiles_total + best - 1) / best);
+  *tiles_per_split = tps;
+  *n_split = (tiles_total + tps - 1) / tps;
+}
 
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
   CUtensorMap maps[7];

@@ -21,7 +21,7 @@ struct Derived {
   long long img_per_head, spec_per_head;
   bool fp32, pads;
   size_t esize;
-  int spec_qtiles, spec_tiles0, spec_tiles_total, spec_split, spec_tps;
+  int spec_tiles0, spec_tiles_total, spec_split, spec_tps;
 };
 
 int validate(const gsa_config* c, Derived* d) {
@@ -66,16 +66,9 @@ int validate(const gsa_config* c, Derived* d) {
   d->esize = d->fp32 ? 4 : 2;
   // special tokens: split the key range so that enough CTAs run
   const long long M = d->spec_per_head;
-  d->spec_qtiles = static_cast<int>((M + 255) / 256);                     // 256 rows per CTA
   d->spec_tiles0 = attn_tc_tiles(M);                                       // 128-key tiles
   d->spec_tiles_total = d->spec_tiles0 + attn_tc_tiles(d->img_per_head);
-  long long want = 148LL * 8 / (static_cast<long long>(c->num_heads) * (d->spec_qtiles > 0 ? d->spec_qtiles : 1));
-  long long maxs = d->spec_tiles_total / 16;
-  long long ns = want < maxs ? want : maxs;
-  if (ns < 1) ns = 1;
-  if (ns > 4096) ns = 4096;
-  d->spec_tps = static_cast<int>((d->spec_tiles_total + ns - 1) / ns);
-  d->spec_split = (d->spec_tiles_total + d->spec_tps - 1) / d->spec_tps;
+  attn_tc_split(c->num_heads, M, d->spec_tiles_total, &d->spec_tps, &d->spec_split);
   return GSA_OK;
 }
 

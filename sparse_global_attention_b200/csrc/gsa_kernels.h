@@ -57,6 +57,9 @@ cudaError_t launch_attn(const AttnArgs& a, bool topk, cudaStream_t st);
 // top-k runs when a.kc > 0 (a.q_lo / a.k_lo required)
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st);
 int attn_tc_tiles(long long n);
+// key-range splits for a launch of n_q query rows per head over tiles_total
+// 128-key tiles (rows of every split are merged by launch_merge)
+void attn_tc_split(int H, long long n_q, int tiles_total, int* tiles_per_split, int* n_split);
 
 struct MergeArgs {
   const float* part_o;

@@ -62,16 +62,10 @@ extern "C" int gsa_special_attention_noalloc(const void* q_spec, const void* k_s
   if (M * num_heads >= (1LL << 31) || N * num_heads >= (1LL << 31)) return GSA_ERR_UNSUPPORTED;
 
   // same split rule as the context path: enough CTAs to fill the GPU
-  const int qtiles = static_cast<int>((M + 255) / 256);
   const int tiles0 = attn_tc_tiles(M);
   const int tiles_total = tiles0 + attn_tc_tiles(N);
-  long long want = 148LL * 8 / (static_cast<long long>(num_heads) * qtiles);
-  long long maxs = tiles_total / 16;
-  long long ns = want < maxs ? want : maxs;
-  if (ns < 1) ns = 1;
-  if (ns > 4096) ns = 4096;
-  const int tps = static_cast<int>((tiles_total + ns - 1) / ns);
-  const int n_split = (tiles_total + tps - 1) / tps;
+  int tps = 0, n_split = 0;
+  attn_tc_split(num_heads, M, tiles_total, &tps, &n_split);
 
   // the partials must fit the static array: otherwise reject, allocate nothing
   const size_t rows = static_cast<size_t>(n_split) * num_heads * M;
