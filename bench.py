@@ -82,6 +82,10 @@ def algorithmic_work(cfg, kc):
                       "bytes": 2.0 * H * slots * d * e + 2.0 * H * slots * d * e + H * R * cfg.topk * 4}
     w["epilogue"] = {"flops": 2.0 * d * d * M * H,
                      "bytes": 3.0 * H * slots * d * e + H * R * d * 4 + H * d * d * e}
+    # selection with the upsample/gate/blend fused: reads Q, every image token's K/V once,
+    # O'_comp and the region lists; writes O_img
+    w["selection_gate"] = {"flops": w["selection"]["flops"] + w["epilogue"]["flops"],
+                           "bytes": 4.0 * H * slots * d * e + H * R * d * 4 + H * R * cfg.topk * 4}
     w["special"] = {"flops": 4.0 * d * Ms * (Ms + M) * H, "bytes": 2.0 * H * (Ms + slots) * d * e + 2.0 * H * Ms * d * e}
     w["special_merge"] = {"flops": 0.0, "bytes": 0.0}
     w["dense"] = {"flops": 4.0 * d * (M + Ms) ** 2 * H, "bytes": 4.0 * H * (slots + Ms) * d * e}

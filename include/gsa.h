@@ -129,19 +129,27 @@ GSA_API int gsa_dense_forward(gsa_ctx *ctx, const void *q, const void *k, const 
  * which: 0 Q_comp, 1 K_comp, 2 V_comp  (context dtype, [H][R][64])
  *        3 O'_comp (fp32, [H][R][64])
  *        4 selected regions (int32, [H][R][topk])
- *        5 O_sel (context dtype, [H][F][pad_h][pad_w][64])
+ *        5 O_sel (context dtype, [H][F][pad_h][pad_w][64]; written only with
+ *          GSA_PROFILE_KEEP_OSEL or when selection and gate run as two kernels)
  *        6, 7 low parts of Q_comp, K_comp: bf16 contexts keep the pooled
  *          value x as bf16 hi = bf16(x) (items 0, 1) plus lo = bf16(x - hi)
  *          ([H][R][64] bf16), fp32 contexts return items 0, 1 again */
 GSA_API int gsa_get_intermediate(gsa_ctx *ctx, int which, void **dev_ptr, size_t *bytes);
 
-/* Per-kernel timing: when enabled, gsa_forward records CUDA events on its
- * stream around each kernel; gsa_get_kernel_times synchronises on the last
- * forward and writes up to `cap` durations in ms (order: pool, compressed +
- * top-k, selection, epilogue, special, special-merge) and their
- * names (static strings).  Returns the number of entries or a negative
- * status. */
-GSA_API int gsa_set_profiling(gsa_ctx *ctx, int enable);
+/* Profiling flags (bitwise or):
+ *   GSA_PROFILE_TIMES      gsa_forward records CUDA events on its stream around
+ *                          each kernel; gsa_get_kernel_times synchronises on the
+ *                          last forward and writes up to `cap` durations in ms
+ *                          (pool, compressed + top-k, selection (with the fused
+ *                          upsample/gate/blend, or followed by a separate
+ *                          epilogue), special, special-merge) and their names
+ *                          (static strings); it returns the number of entries
+ *                          or a negative status.
+ *   GSA_PROFILE_KEEP_OSEL  keep O_sel in the workspace (gsa_get_intermediate 5);
+ *                          the fused selection kernel otherwise never writes it. */
+#define GSA_PROFILE_TIMES     1
+#define GSA_PROFILE_KEEP_OSEL 2
+GSA_API int gsa_set_profiling(gsa_ctx *ctx, int flags);
 GSA_API int gsa_get_kernel_times(gsa_ctx *ctx, float *ms, const char **names, int cap);
 
 /* Synchronise the context's last stream and return (then clear) the device

@@ -19,6 +19,7 @@ GSA_OK = 0
 GSA_BF16, GSA_FP32 = 0, 1
 GSA_GATE_LEARNED, GSA_GATE_COMP_ONLY, GSA_GATE_SEL_ONLY = 0, 1, 2
 GATE_MODES = {"learned": 0, "comp_only": 1, "sel_only": 2}
+GSA_PROFILE_TIMES, GSA_PROFILE_KEEP_OSEL = 1, 2
 EXPORTED = ("gsa_create", "gsa_workspace_bytes", "gsa_forward", "gsa_dense_forward",
             "gsa_get_intermediate", "gsa_set_profiling", "gsa_get_kernel_times",
             "gsa_get_status", "gsa_strerror", "gsa_destroy", "gsa_special_attention_noalloc")
@@ -142,8 +143,10 @@ def gsa_get_intermediate(ctx, which: int):
     return p.value, n.value
 
 
-def gsa_set_profiling(ctx, enable: bool):
-    _check(load_library().gsa_set_profiling(ctx, 1 if enable else 0), "gsa_set_profiling")
+def gsa_set_profiling(ctx, flags):
+    """flags: GSA_PROFILE_TIMES (per-kernel CUDA-event timing) | GSA_PROFILE_KEEP_OSEL;
+    True/False mean GSA_PROFILE_TIMES / 0."""
+    _check(load_library().gsa_set_profiling(ctx, int(flags)), "gsa_set_profiling")
 
 
 def gsa_get_kernel_times(ctx, cap: int = 16):

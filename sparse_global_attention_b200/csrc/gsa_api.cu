@@ -143,10 +143,10 @@ struct Prof {
   cudaStream_t st;
   Prof(gsa_ctx* c, cudaStream_t s) : ctx(c), st(s) {
     ctx->n_ev = 0;
-    if (ctx->profiling) cudaEventRecord(ctx->ev[ctx->n_ev++], st);
+    if (ctx->profiling & GSA_PROFILE_TIMES) cudaEventRecord(ctx->ev[ctx->n_ev++], st);
   }
   void mark(const char* name) {
-    if (ctx->profiling && ctx->n_ev < MAX_EVENTS) {
+    if ((ctx->profiling & GSA_PROFILE_TIMES) && ctx->n_ev < MAX_EVENTS) {
       ctx->ev_names[ctx->n_ev - 1] = name;
       cudaEventRecord(ctx->ev[ctx->n_ev++], st);
     }
@@ -288,7 +288,7 @@ int gsa_forward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void* 
   }
   prof.mark("comp_attn_topk");
 
-  // K3 selection
+  // K3 selection (+ K4 upsample/gate/blend, fused for bf16)
   SelArgs sa;
   sa.q_img = q_img; sa.k_img = k_img; sa.v_img = v_img; sa.k_spec = k_spec; sa.v_spec = v_spec;
   sa.idx = c->at<int>(c->L.idx); sa.o_sel = c->ws + c->L.osel;
@@ -296,16 +296,21 @@ int gsa_forward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void* 
   sa.g = g; sa.scale_log2 = scale * LOG2E; sa.n_fixed = cf.num_fixed_frames;
   for (int i = 0; i < cf.num_fixed_frames; ++i) sa.fixed[i] = c->fixed[i];
   sa.err = err;
-  if (launch_sel(sa, d.fp32, st) != cudaSuccess) return GSA_ERR_CUDA;
-  prof.mark("selection");
-
-  // K4 upsample + gate + blend
   EpiArgs ea;
   ea.q_img = q_img; ea.o_sel = c->ws + c->L.osel; ea.o_comp = c->at<float>(c->L.ocomp);
   ea.w_g = w_g; ea.o_img = o_img; ea.H = H; ea.F = cf.num_frames; ea.R = d.R; ea.rpf = d.rpf;
   ea.s = cf.pool_s; ea.g = g; ea.gate_mode = cf.gate_mode;
-  if (launch_epilogue(ea, d.fp32, st) != cudaSuccess) return GSA_ERR_CUDA;
-  prof.mark("epilogue");
+  if (!d.fp32) {
+    // O_sel is written only when the caller asked to keep intermediates
+    if (!(c->profiling & GSA_PROFILE_KEEP_OSEL)) sa.o_sel = nullptr;
+    if (launch_sel_fused(sa, ea, st) != cudaSuccess) return GSA_ERR_CUDA;
+    prof.mark("selection_gate");
+  } else {
+    if (launch_sel(sa, d.fp32, st) != cudaSuccess) return GSA_ERR_CUDA;
+    prof.mark("selection");
+    if (launch_epilogue(ea, d.fp32, st) != cudaSuccess) return GSA_ERR_CUDA;
+    prof.mark("epilogue");
+  }
 
   // K5 special tokens over every token
   if (cf.num_special > 0) {
@@ -429,14 +434,14 @@ int gsa_get_intermediate(gsa_ctx* c, int which, void** dev_ptr, size_t* bytes) {
 
 int gsa_set_profiling(gsa_ctx* c, int enable) {
   if (!c) return GSA_ERR_INVALID_ARG;
-  c->profiling = enable ? 1 : 0;
+  c->profiling = enable;
   c->n_ev = 0;
   return GSA_OK;
 }
 
 int gsa_get_kernel_times(gsa_ctx* c, float* ms, const char** names, int cap) {
   if (!c || cap < 0) return -GSA_ERR_INVALID_ARG;
-  if (!c->profiling || c->n_ev < 2) return 0;
+  if (!(c->profiling & GSA_PROFILE_TIMES) || c->n_ev < 2) return 0;
   DeviceGuard dg(c->device);
   if (cudaEventSynchronize(c->ev[c->n_ev - 1]) != cudaSuccess) return -GSA_ERR_CUDA;
   int n = 0;

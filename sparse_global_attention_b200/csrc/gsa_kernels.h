@@ -103,6 +103,10 @@ struct EpiArgs {
 };
 cudaError_t launch_epilogue(const EpiArgs& a, bool fp32, cudaStream_t st);
 
+// ---- K3 + K4 fused (bf16, s in {1, 2, 4}): selection attention, then the
+// upsample/gate/blend of the window's tokens in the same kernel -------------
+cudaError_t launch_sel_fused(const SelArgs& a, const EpiArgs& ep, cudaStream_t st);
+
 // ---- fp32 (SIMT) variants for fp32 contexts ---------------------------------
 struct AttnF32Args {
   const float* q; long long q_hs; int n_q; int q_mask;

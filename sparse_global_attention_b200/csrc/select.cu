@@ -8,7 +8,8 @@
 // key set also holds a fixed global context: every token of the reference
 // frame and of the frames sampled every 100 frames.
 //
-// bf16 path: one warp per window (s*s <= 16 queries fill one m16 MMA tile);
+// bf16 path (with the K4 epilogue fused in: O_img is written directly): one
+// warp per window (s*s <= 16 queries fill one m16 MMA tile);
 // 4 windows per CTA, neighbours in raster order so their overlapping region
 // choices meet in L2.  Each warp gathers its keys 32 at a time (the tokens of
 // the selected regions, then the fixed context) into its own double-buffered
@@ -72,8 +73,19 @@ __device__ __forceinline__ bool key_src(const SelArgs& a, const int2* rb, int p,
   return a.g.img_valid(o - a.g.ns);
 }
 
-template <int S>
-__global__ void __launch_bounds__(SEL_WARPS * 32) sel_kernel_bf16(const SelArgs a) {
+__device__ __forceinline__ float sigmoid_fast(float x) {
+  const float e = ex2(fminf(-x * LOG2E, 126.f));
+  return __fdividef(1.f, 1.f + e);
+}
+
+// GATE: the window's outputs go straight through the K4 epilogue (nearest
+// upsample of O'_comp, g = sigmoid(W_g q), blend) and O_img is written; O_sel
+// itself is written only when a.o_sel is set.  G = Q W_g^T reuses the
+// window's Q fragments; W_g's B fragments are 32-bit loads of its rows (L1);
+// g is computed before the key loop and held as bf16 pairs (relative error
+// 2^-9 of g, below the bf16 rounding of the output).
+template <int S, bool GATE>
+__global__ void __launch_bounds__(SEL_WARPS * 32) sel_kernel_bf16(const SelArgs a, const EpiArgs ep) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3, mi = lane >> 3, lr = lane & 7;
@@ -153,6 +165,31 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) sel_kernel_bf16(const SelArgs 
   for (int ks = 0; ks < 4; ++ks)
     ldsm_x4(sQ + swz(lr + 8 * (mi & 1), 2 * ks + (mi >> 1)), qf[ks][0], qf[ks][1], qf[ks][2],
             qf[ks][3]);
+
+  // gate (fused epilogue): g = sigmoid(Q W_g^T) now, while the first keys are
+  // in flight; kept as bf16 pairs (channel pair of each accumulator element)
+  uint32_t gp[8][2];
+  if constexpr (GATE) {
+    const float gfix = ep.gate_mode == 1 ? 1.f : 0.f;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) gp[nt][0] = gp[nt][1] = pack_bf16(gfix, gfix);
+    if (ep.gate_mode == 0) {
+      const __nv_bfloat16* wg = reinterpret_cast<const __nv_bfloat16*>(ep.w_g) + static_cast<long long>(h) * D * D;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        float ga[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const __nv_bfloat16* wr = wg + (8 * nt + g) * D + 16 * ks + 2 * t;
+          const uint32_t b0 = __ldg(reinterpret_cast<const unsigned int*>(wr));
+          const uint32_t b1 = __ldg(reinterpret_cast<const unsigned int*>(wr + 8));
+          mma_bf16(ga, qf[ks], b0, b1);
+        }
+        gp[nt][0] = pack_bf16(sigmoid_fast(ga[0]), sigmoid_fast(ga[1]));
+        gp[nt][1] = pack_bf16(sigmoid_fast(ga[2]), sigmoid_fast(ga[3]));
+      }
+    }
+  }
 
   float o[8][4];
 #pragma unroll
@@ -237,7 +274,9 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) sel_kernel_bf16(const SelArgs 
   }
   cp_async_wait<0>();
 
-  __nv_bfloat16* oh = reinterpret_cast<__nv_bfloat16*>(a.o_sel) + h * img_hs;
+  __nv_bfloat16* oh = a.o_sel ? reinterpret_cast<__nv_bfloat16*>(a.o_sel) + h * img_hs : nullptr;
+  __nv_bfloat16* ih = GATE ? reinterpret_cast<__nv_bfloat16*>(ep.o_img) + h * img_hs : nullptr;
+  const float* cr = GATE ? ep.o_comp + (static_cast<long long>(h) * a.R + r) * D : nullptr;
 #pragma unroll
   for (int rr = 0; rr < 2; ++rr) {
     l[rr] += __shfl_xor_sync(0xffffffffu, l[rr], 1);
@@ -249,9 +288,22 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) sel_kernel_bf16(const SelArgs 
     const float inv = (qv && l[rr] > 0.f) ? 1.f / l[rr] : 0.f;
     const long long tok = (static_cast<long long>(f) * a.g.Hp + y) * a.g.Wp + x;
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-      *reinterpret_cast<uint32_t*>(oh + tok * D + 8 * nt + 2 * t) =
-          pack_bf16(o[nt][2 * rr] * inv, o[nt][2 * rr + 1] * inv);
+    for (int nt = 0; nt < 8; ++nt) {
+      const int c = 8 * nt + 2 * t;
+      const float s0 = o[nt][2 * rr] * inv, s1 = o[nt][2 * rr + 1] * inv;
+      if (oh) *reinterpret_cast<uint32_t*>(oh + tok * D + c) = pack_bf16(s0, s1);
+      if constexpr (GATE) {
+        float out0 = 0.f, out1 = 0.f;
+        if (qv) {
+          const float2 gg = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gp[nt][rr]));
+          const float g0 = gg.x, g1 = gg.y;
+          const float2 oc = __ldg(reinterpret_cast<const float2*>(cr + c));
+          out0 = g0 * oc.x + (1.f - g0) * s0;
+          out1 = g1 * oc.y + (1.f - g1) * s1;
+        }
+        *reinterpret_cast<uint32_t*>(ih + tok * D + c) = pack_bf16(out0, out1);
+      }
+    }
   }
 }
 
@@ -326,15 +378,36 @@ cudaError_t launch_sel_s(const SelArgs& a, bool fp32, cudaStream_t st) {
     sel_kernel_f32<S><<<static_cast<unsigned>((n + 127) / 128), 128, 0, st>>>(a);
   } else {
     const int sm = SEL_WARPS * SEL_WARP_SMEM;
-    cudaError_t e = cudaFuncSetAttribute(sel_kernel_bf16<S>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    cudaError_t e = cudaFuncSetAttribute(sel_kernel_bf16<S, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
     if (e != cudaSuccess) return e;
     const long long w = static_cast<long long>(a.H) * a.R;
-    sel_kernel_bf16<S><<<static_cast<unsigned>((w + SEL_WARPS - 1) / SEL_WARPS), SEL_WARPS * 32, sm, st>>>(a);
+    EpiArgs none;
+    memset(&none, 0, sizeof(none));
+    sel_kernel_bf16<S, false><<<static_cast<unsigned>((w + SEL_WARPS - 1) / SEL_WARPS), SEL_WARPS * 32, sm, st>>>(a, none);
   }
   return cudaGetLastError();
 }
 
+template <int S>
+cudaError_t launch_sel_fused_s(const SelArgs& a, const EpiArgs& ep, cudaStream_t st) {
+  const int sm = SEL_WARPS * SEL_WARP_SMEM;
+  cudaError_t e = cudaFuncSetAttribute(sel_kernel_bf16<S, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+  if (e != cudaSuccess) return e;
+  const long long w = static_cast<long long>(a.H) * a.R;
+  sel_kernel_bf16<S, true><<<static_cast<unsigned>((w + SEL_WARPS - 1) / SEL_WARPS), SEL_WARPS * 32, sm, st>>>(a, ep);
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_sel_fused(const SelArgs& a, const EpiArgs& ep, cudaStream_t st) {
+  switch (a.s) {
+    case 1: return launch_sel_fused_s<1>(a, ep, st);
+    case 2: return launch_sel_fused_s<2>(a, ep, st);
+    case 4: return launch_sel_fused_s<4>(a, ep, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
 
 cudaError_t launch_sel(const SelArgs& a, bool fp32, cudaStream_t st) {
   switch (a.s) {

@@ -42,6 +42,7 @@ def assert_close(name, got, want, cfg, mask=None):
 def run_gpu(cfg, x, gate_mode="learned", topk=None):
     """One gsa_forward through the C ABI; returns outputs and intermediates on the host."""
     layer = gsa.GSALayer.from_workload(cfg, gate_mode=gate_mode, topk=topk)
+    gsa.gsa_set_profiling(layer.ctx, gsa.GSA_PROFILE_KEEP_OSEL)   # keep O_sel for the checks
     k = cfg.topk if topk is None else topk
     R = cfg.num_regions
     H = cfg.num_heads
