@@ -159,6 +159,17 @@ GSA_API int gsa_get_status(gsa_ctx *ctx);
 /* Static text for a status code. */
 GSA_API const char *gsa_strerror(int code);
 
+/* Failure-detection self-test (the notes describe no counterpart).  Launches,
+ * asynchronously on `stream`, one CTA that waits on an mbarrier nothing ever
+ * completes, with the same bounded polling as the layer's kernels; the wait
+ * gives up after limit_us microseconds of global time (1 .. 1,000,000) and
+ * records GSA_ERR_DEVICE_TIMEOUT in the context's error word.  Nothing faults
+ * or hangs, and the context stays usable: gsa_get_status then returns (and
+ * clears) GSA_ERR_DEVICE_TIMEOUT, and later calls run normally.  Returns
+ * GSA_ERR_INVALID_ARG for a NULL context or a limit out of range,
+ * GSA_ERR_CUDA if the launch fails. */
+GSA_API int gsa_debug_expire_wait(gsa_ctx *ctx, unsigned int limit_us, void *stream);
+
 /* Free the workspace and the context; NULL is accepted. */
 GSA_API void gsa_destroy(gsa_ctx *ctx);
 

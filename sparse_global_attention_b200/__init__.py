@@ -22,7 +22,8 @@ GATE_MODES = {"learned": 0, "comp_only": 1, "sel_only": 2}
 GSA_PROFILE_TIMES, GSA_PROFILE_KEEP_OSEL = 1, 2
 EXPORTED = ("gsa_create", "gsa_workspace_bytes", "gsa_forward", "gsa_dense_forward",
             "gsa_get_intermediate", "gsa_set_profiling", "gsa_get_kernel_times",
-            "gsa_get_status", "gsa_strerror", "gsa_destroy", "gsa_special_attention_noalloc")
+            "gsa_get_status", "gsa_strerror", "gsa_destroy", "gsa_special_attention_noalloc",
+            "gsa_debug_expire_wait")
 
 
 class gsa_config(ctypes.Structure):
@@ -160,6 +161,15 @@ def gsa_get_kernel_times(ctx, cap: int = 16):
 
 def gsa_get_status(ctx) -> int:
     return load_library().gsa_get_status(ctx)
+
+
+def gsa_debug_expire_wait(ctx, limit_us: int, stream=None):
+    """Failure-detection self-test: a device wait that runs out after limit_us
+    and records GSA_ERR_DEVICE_TIMEOUT in the context's error word."""
+    fn = load_library().gsa_debug_expire_wait
+    fn.argtypes = [ctypes.c_void_p, ctypes.c_uint, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    _check(fn(ctx, int(limit_us), stream or None), "gsa_debug_expire_wait")
 
 
 def gsa_strerror(code: int) -> str:

@@ -454,6 +454,15 @@ int gsa_get_kernel_times(gsa_ctx* c, float* ms, const char** names, int cap) {
   return n;
 }
 
+int gsa_debug_expire_wait(gsa_ctx* c, unsigned int limit_us, void* stream) {
+  if (!c || limit_us < 1 || limit_us > 1000000) return GSA_ERR_INVALID_ARG;
+  DeviceGuard dg(c->device);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (launch_expire_wait(c->at<int>(c->L.err), 1000ull * limit_us, st) != cudaSuccess) return GSA_ERR_CUDA;
+  c->last_stream = st;
+  return GSA_OK;
+}
+
 int gsa_get_status(gsa_ctx* c) {
   if (!c) return GSA_ERR_INVALID_ARG;
   DeviceGuard dg(c->device);

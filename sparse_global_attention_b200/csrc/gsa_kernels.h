@@ -118,4 +118,9 @@ struct AttnF32Args {
 };
 cudaError_t launch_attn_f32(const AttnF32Args& a, bool topk, cudaStream_t st);
 
+// ---- failure-detection self-test ---------------------------------------------
+// one CTA waits on an mbarrier that nothing completes, gives up after limit_ns
+// of global time and records the timeout code in *err
+cudaError_t launch_expire_wait(int* err, unsigned long long limit_ns, cudaStream_t st);
+
 }  // namespace gsa

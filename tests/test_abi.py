@@ -1,5 +1,6 @@
 """The C ABI without a GPU: the library loads, exports every entry point the
 header declares, and rejects invalid configurations on the host."""
+import ctypes
 import os
 import re
 
@@ -76,4 +77,7 @@ def test_strerror_and_null_safety():
     lib = gsa.load_library()
     lib.gsa_destroy(None)                         # NULL-safe
     assert lib.gsa_get_status(None) == 1
+    fn = lib.gsa_debug_expire_wait
+    fn.argtypes = [ctypes.c_void_p, ctypes.c_uint, ctypes.c_void_p]
+    assert fn(None, 1000, None) == 1              # NULL context: GSA_ERR_INVALID_ARG, nothing launched
     assert lib.gsa_forward(None, *([None] * 11)) == 1
