@@ -437,6 +437,33 @@ def run_b200(args, cfg, rank, world, local, dist):
                           f"all windows and heads; BLAS {blas}; {cores} cores visible")}
 
     layer.close()
+
+    # ---- ablation variants of the notes' table, same inputs (optional) -------------
+    ablations = None
+    if args.ablations:
+        ablations = {}
+        specs = [("no_comp_value", dict(variant="no_comp_value")), ("no_selection", dict(variant="no_selection")),
+                 ("top8", dict(topk=8)), ("top16", dict(topk=16)), ("top64", dict(topk=64))]
+        for name, kw in specs:
+            lay = gsa.GSALayer.from_workload(cfg, **kw)
+            for _ in range(2):
+                lay.forward(x, out=out)
+            torch.cuda.synchronize()
+            barrier()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            for _ in range(3):
+                lay.forward(x, out=out)
+            a1.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            st = lay.status()
+            lay.close()
+            if st != 0:
+                raise RuntimeError(f"device status {st} in ablation {name}: {gsa.gsa_strerror(st)}")
+            ams = max_over_ranks(a0.elapsed_time(a1) / 3, dist, dev)
+            ablations[name] = {"ms": round(ams, 3), "vs_full": round(ams / ms, 3)}
+
     if rank != 0:
         return None
     line = {
@@ -452,6 +479,8 @@ def run_b200(args, cfg, rank, world, local, dist):
         "kernels": kernels, "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(), "e2e": e2e, "cpu_baseline": cpu,
     }
+    if ablations is not None:
+        line["ablations"] = ablations
     return line
 
 
@@ -465,6 +494,9 @@ def main():
     ap.add_argument("--dense", default="full", choices=["full", "off"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ablations", action="store_true",
+                    help="also time the layer variants of the ablation table (no compressed value, "
+                         "no selection, top-8/16/64) on the same inputs")
     ap.add_argument("--cpu-windows", type=int, default=2048)
     ap.add_argument("--ref-windows", type=int, default=512)
     args = ap.parse_args()

@@ -67,6 +67,20 @@ extern "C" {
 #define GSA_MAX_TOPK         64
 #define GSA_MAX_FIXED_FRAMES 16
 
+/* Layer variants of the notes' ablation study ("消融实验", rows (1) and (2)).
+ * They change what is computed, not only the output:
+ *   GSA_VARIANT_FULL           the layer as described: O_img = g O_comp + (1-g) O_sel
+ *   GSA_VARIANT_NO_COMP_VALUE  "移除压缩分支 Value": the compressed branch keeps only
+ *                              its guide (S_guide and the top-k; no V_comp, no P V),
+ *                              O_img = O_sel (the gate has nothing to blend with)
+ *   GSA_VARIANT_NO_SELECTION   "移除选择分支": no top-k and no selection branch,
+ *                              O_img = Upsample(O'_comp); sel_idx_out must be NULL
+ * gate_mode is ignored by the two ablation variants; special tokens are
+ * computed as in the full layer. */
+#define GSA_VARIANT_FULL          0
+#define GSA_VARIANT_NO_COMP_VALUE 1
+#define GSA_VARIANT_NO_SELECTION  2
+
 typedef struct gsa_ctx gsa_ctx;
 
 typedef struct {
@@ -78,7 +92,7 @@ typedef struct {
                               camera tokens removed, pi^3 adaptation)             */
     int num_heads;         /* H >= 1                                              */
     int head_dim;          /* must be 64                                          */
-    int pool_s;            /* s in {1, 2, 4, 8} (bf16 path: {2, 4})               */
+    int pool_s;            /* s in {1, 2, 4, 8} (bf16 path: {1, 2, 4})            */
     int topk;              /* regions per compressed query, 1..min(64, candidates) */
     int dtype;             /* GSA_BF16 or GSA_FP32                                */
     const int *fixed_frames; /* VGGT fixed global context frames (copied at
@@ -86,6 +100,7 @@ typedef struct {
     int num_fixed_frames;
     int gate_mode;         /* GSA_GATE_*                                          */
     float softmax_scale;   /* 0 => 1/sqrt(head_dim)                               */
+    int variant;           /* GSA_VARIANT_* (0 = the full layer)                  */
 } gsa_config;
 
 /* Validate `cfg` and create a context on the current CUDA device; allocates

@@ -19,6 +19,7 @@ GSA_OK = 0
 GSA_BF16, GSA_FP32 = 0, 1
 GSA_GATE_LEARNED, GSA_GATE_COMP_ONLY, GSA_GATE_SEL_ONLY = 0, 1, 2
 GATE_MODES = {"learned": 0, "comp_only": 1, "sel_only": 2}
+VARIANTS = {"full": 0, "no_comp_value": 1, "no_selection": 2}
 GSA_PROFILE_TIMES, GSA_PROFILE_KEEP_OSEL = 1, 2
 EXPORTED = ("gsa_create", "gsa_workspace_bytes", "gsa_forward", "gsa_dense_forward",
             "gsa_get_intermediate", "gsa_set_profiling", "gsa_get_kernel_times",
@@ -34,6 +35,7 @@ class gsa_config(ctypes.Structure):
         ("topk", ctypes.c_int), ("dtype", ctypes.c_int),
         ("fixed_frames", ctypes.POINTER(ctypes.c_int)), ("num_fixed_frames", ctypes.c_int),
         ("gate_mode", ctypes.c_int), ("softmax_scale", ctypes.c_float),
+        ("variant", ctypes.c_int),
     ]
 
 
@@ -88,7 +90,7 @@ def _check(rc: int, what: str):
 def make_config(*, num_frames, grid_h, grid_w, pad_h=None, pad_w=None, num_special=0,
                 num_heads=1, head_dim=64, pool_s=4, topk=32, dtype="bf16",
                 fixed_frames: Sequence[int] = (), gate_mode="learned",
-                softmax_scale=0.0) -> gsa_config:
+                softmax_scale=0.0, variant="full") -> gsa_config:
     c = gsa_config()
     c.num_frames, c.grid_h, c.grid_w = num_frames, grid_h, grid_w
     c.pad_h = grid_h if pad_h is None else pad_h
@@ -102,6 +104,7 @@ def make_config(*, num_frames, grid_h, grid_w, pad_h=None, pad_w=None, num_speci
     c.num_fixed_frames = len(fixed_frames)
     c.gate_mode = GATE_MODES[gate_mode] if isinstance(gate_mode, str) else int(gate_mode)
     c.softmax_scale = float(softmax_scale)
+    c.variant = VARIANTS[variant] if isinstance(variant, str) else int(variant)
     return c
 
 

@@ -53,12 +53,13 @@ constexpr float RESCALE_LOG2 = 8.f;      // rescale O when the max grows by > 2^
 constexpr uint32_t IDESC_QK = idesc_bf16(128, 128, false);
 constexpr uint32_t IDESC_PV = idesc_bf16(128, 64, true);
 
-template <int KC>
+// GO (guide only, the "no compressed value" ablation): S and the top-k, no P V.
+template <int KC, bool GO = false>
 struct Lay {
   static constexpr bool TOPK = KC > 0;
   static constexpr int NST = 3;                        // K/V ring depth
   static constexpr int QT = TOPK ? 2 : 1;              // tiles per query tile (hi[, lo])
-  static constexpr int KT = TOPK ? 3 : 2;              // tiles per stage: K hi, [K lo], V
+  static constexpr int KT = GO ? 2 : (TOPK ? 3 : 2);   // tiles per stage: K hi, [K lo], [V]
   static constexpr int KV = 2 * QT * TILE;             // Q_i hi at i*TILE, lo at (2+i)*TILE
   static constexpr int STAGE = KT * TILE;
   static constexpr int BAR = KV + NST * STAGE;
@@ -225,13 +226,13 @@ __device__ __forceinline__ void topk_insert(float (&ts)[KC > 0 ? KC : 1], int (&
   }
 }
 
-template <int KC>
+template <int KC, bool GO>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qlo,
                    const __grid_constant__ CUtensorMap tm_k0, const __grid_constant__ CUtensorMap tm_v0,
                    const __grid_constant__ CUtensorMap tm_k1, const __grid_constant__ CUtensorMap tm_v1,
                    const __grid_constant__ CUtensorMap tm_klo, const AttnArgs a) {
-  using L = Lay<KC>;
+  using L = Lay<KC, GO>;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the 128B-swizzle atoms
   const uint32_t raw = smem_u32(smem_raw);
@@ -301,7 +302,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           mbar_expect_tx(bars.full(s), L::KT * TILE);
           tma_load_2d(st, seg ? &tm_k1 : &tm_k0, 0, y, bars.full(s));
           if constexpr (L::TOPK) tma_load_2d(st + TILE, &tm_klo, 0, y, bars.full(s));
-          tma_load_2d(st + (L::KT - 1) * TILE, seg ? &tm_v1 : &tm_v0, 0, y, bars.full(s));
+          if constexpr (!GO) tma_load_2d(st + (L::KT - 1) * TILE, seg ? &tm_v1 : &tm_v0, 0, y, bars.full(s));
         }
         __syncwarp();
         ++issued;
@@ -355,7 +356,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             __syncwarp();
           }
-          if (j > 0) {
+          if (!GO && j > 0) {
             // O_i += P_{i,j-1} V_{j-1}: P read from TMEM (TS form), V MN-major
             ok = __all_sync(0xffffffffu, mbar_wait(bars.p_full(i), (j - 1) & 1, a.err));
             if (!ok) break;
@@ -492,6 +493,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
           }
         }
+        if constexpr (GO) {
+          // guide only: S_i goes straight back, nothing else to compute
+          tc_fence_before();
+          warp_arrive(bars.s_free(qi));
+          continue;
+        }
         rescale(mx, m, l, j, qi, tO, bars, a.err, ok, sl2);
         if (!ok) break;
         // pass 2: P = exp2((S - m) * scale * log2e) in bf16 to shared memory; S_i
@@ -535,11 +542,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       warp_arrive(bars.p_full(qi));
     }
     // ---- epilogue: O_i row from TMEM ----------------------------------------
-    if (ok && ntile > 0) ok = mbar_wait(bars.pv_done(qi), (ntile - 1) & 1, a.err);
+    if (!GO && ok && ntile > 0) ok = mbar_wait(bars.pv_done(qi), (ntile - 1) & 1, a.err);
     ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
     float o[64];
-    if (ok && ntile > 0) {
+    if (!GO && ok && ntile > 0) {
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t v[32];
@@ -553,7 +560,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int e = 0; e < 64; ++e) o[e] = 0.f;
     }
     if (row < a.n_q) {
-      if (a.n_split == 1) {
+      if (GO) {
+        // guide only: no attention output
+      } else if (a.n_split == 1) {
         float inv = l > 0.f ? 1.f / l : 0.f;
         if (a.q_mask != MASK_NONE && !key_valid(a.q_mask, a.g, row)) inv = 0.f;
         const long long base = h * a.o_hs + static_cast<long long>(row) * D;
@@ -626,14 +635,19 @@ bool make_map(CUtensorMap* m, const void* base, long long rows) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int KC>
+template <int KC, bool GO>
 cudaError_t launch_kc(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t st) {
-  const int sm = Lay<KC>::BYTES;
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<KC>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+  const int sm = Lay<KC, GO>::BYTES;
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<KC, GO>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
   if (e != cudaSuccess) return e;
   dim3 grid((a.n_q + 2 * TBM - 1) / (2 * TBM), a.n_split, a.H);
-  attn_tc_kernel<KC><<<grid, NTHREADS, sm, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], a);
+  attn_tc_kernel<KC, GO><<<grid, NTHREADS, sm, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], a);
   return cudaGetLastError();
+}
+
+template <int KC>
+cudaError_t launch_kc2(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t st) {
+  return a.guide_only ? launch_kc<KC, true>(a, maps, st) : launch_kc<KC, false>(a, maps, st);
 }
 
 }  // namespace
@@ -675,19 +689,21 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
   if (!make_map(&maps[0], a.q, H * a.n_q)) return cudaErrorInvalidValue;
   maps[1] = maps[0];
   if (a.kc > 0 && !make_map(&maps[1], a.q_lo, H * a.n_q)) return cudaErrorInvalidValue;
-  if (!make_map(&maps[2], a.k[0], H * a.n_k[0]) || !make_map(&maps[3], a.v[0], H * a.n_k[0]))
-    return cudaErrorInvalidValue;
+  if (a.guide_only && (a.kc == 0 || a.nseg != 1 || a.n_split != 1)) return cudaErrorInvalidValue;
+  if (!make_map(&maps[2], a.k[0], H * a.n_k[0])) return cudaErrorInvalidValue;
+  maps[3] = maps[2];                       // guide only: V is never loaded
+  if (!a.guide_only && !make_map(&maps[3], a.v[0], H * a.n_k[0])) return cudaErrorInvalidValue;
   maps[4] = maps[2];
   maps[5] = maps[3];
   if (a.nseg > 1 && (!make_map(&maps[4], a.k[1], H * a.n_k[1]) || !make_map(&maps[5], a.v[1], H * a.n_k[1])))
     return cudaErrorInvalidValue;
   maps[6] = maps[2];
   if (a.kc > 0 && !make_map(&maps[6], a.k_lo, H * a.n_k[0])) return cudaErrorInvalidValue;
-  if (a.kc == 0) return launch_kc<0>(a, maps, st);
-  if (a.kc <= 8) return launch_kc<8>(a, maps, st);
-  if (a.kc <= 16) return launch_kc<16>(a, maps, st);
-  if (a.kc <= 32) return launch_kc<32>(a, maps, st);
-  if (a.kc <= 64) return launch_kc<64>(a, maps, st);
+  if (a.kc == 0) return launch_kc<0, false>(a, maps, st);
+  if (a.kc <= 8) return launch_kc2<8>(a, maps, st);
+  if (a.kc <= 16) return launch_kc2<16>(a, maps, st);
+  if (a.kc <= 32) return launch_kc2<32>(a, maps, st);
+  if (a.kc <= 64) return launch_kc2<64>(a, maps, st);
   return cudaErrorInvalidValue;
 }
 

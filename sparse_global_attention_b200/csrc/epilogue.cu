@@ -55,7 +55,7 @@ __global__ void __launch_bounds__(EPI_WARPS * 32) epi_kernel_bf16(const EpiArgs 
   __syncthreads();
 
   const __nv_bfloat16* qh = reinterpret_cast<const __nv_bfloat16*>(a.q_img) + h * img_hs;
-  const __nv_bfloat16* sh = reinterpret_cast<const __nv_bfloat16*>(a.o_sel) + h * img_hs;
+  const __nv_bfloat16* sh = a.o_sel ? reinterpret_cast<const __nv_bfloat16*>(a.o_sel) + h * img_hs : nullptr;
   const float* ch = a.o_comp + static_cast<long long>(h) * a.R * D;
   __nv_bfloat16* oh = reinterpret_cast<__nv_bfloat16*>(a.o_img) + h * img_hs;
   const uint32_t sQ = smem_u32(sQall[warp]);
@@ -110,8 +110,10 @@ __global__ void __launch_bounds__(EPI_WARPS * 32) epi_kernel_bf16(const EpiArgs 
           if (a.gate_mode == 1) { g0 = g1 = 1.f; }
           else if (a.gate_mode == 2) { g0 = g1 = 0.f; }
           else { g0 = sigmoid_fast(gacc[nt][2 * rr]); g1 = sigmoid_fast(gacc[nt][2 * rr + 1]); }
-          const float2 oc = __ldg(reinterpret_cast<const float2*>(cp + c));
-          const float2 os = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(sp + c));
+          // a forced gate never reads the branch it drops (it may not have been computed)
+          const float2 oc = a.gate_mode == 2 ? make_float2(0.f, 0.f) : __ldg(reinterpret_cast<const float2*>(cp + c));
+          const float2 os = a.gate_mode == 1 ? make_float2(0.f, 0.f)
+                                             : __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(sp + c));
           out0 = g0 * oc.x + (1.f - g0) * os.x;
           out1 = g1 * oc.y + (1.f - g1) * os.y;
         }
@@ -141,8 +143,9 @@ __global__ void __launch_bounds__(256) epi_kernel_f32(const EpiArgs a) {
   float gv = 1.f / (1.f + expf(-gsum));
   if (a.gate_mode == 1) gv = 1.f;
   if (a.gate_mode == 2) gv = 0.f;
-  const float oc = a.o_comp[(static_cast<long long>(h) * a.R + reg) * D + c];
-  const float os = reinterpret_cast<const float*>(a.o_sel)[hn * D + c];
+  // a forced gate never reads the branch it drops (it may not have been computed)
+  const float oc = a.gate_mode == 2 ? 0.f : a.o_comp[(static_cast<long long>(h) * a.R + reg) * D + c];
+  const float os = a.gate_mode == 1 ? 0.f : reinterpret_cast<const float*>(a.o_sel)[hn * D + c];
   *out = gv * oc + (1.f - gv) * os;
 }
 

@@ -34,6 +34,7 @@ int validate(const gsa_config* c, Derived* d) {
   if (c->num_fixed_frames < 0 || (c->num_fixed_frames > 0 && !c->fixed_frames))
     return GSA_ERR_INVALID_ARG;
   if (c->num_fixed_frames > GSA_MAX_FIXED_FRAMES) return GSA_ERR_UNSUPPORTED;
+  if (c->variant < GSA_VARIANT_FULL || c->variant > GSA_VARIANT_NO_SELECTION) return GSA_ERR_INVALID_ARG;
   if (!(c->softmax_scale >= 0.f) || isinf(c->softmax_scale)) return GSA_ERR_INVALID_ARG;
   if (c->head_dim != 64) return GSA_ERR_SHAPE;
   const int s = c->pool_s;
@@ -225,7 +226,13 @@ int gsa_forward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void* 
   const gsa_config& cf = c->cfg;
   const Derived& d = c->d;
   if (cf.num_special > 0 && (!q_spec || !k_spec || !v_spec || !o_spec)) return GSA_ERR_INVALID_ARG;
-  if (cf.gate_mode == GSA_GATE_LEARNED && !w_g) return GSA_ERR_INVALID_ARG;
+  // the ablation variants fix the blend: no compressed value -> O_sel, no selection -> O_comp
+  const int gate = cf.variant == GSA_VARIANT_NO_COMP_VALUE ? GSA_GATE_SEL_ONLY
+                   : cf.variant == GSA_VARIANT_NO_SELECTION ? GSA_GATE_COMP_ONLY
+                                                            : cf.gate_mode;
+  const bool no_sel = cf.variant == GSA_VARIANT_NO_SELECTION;
+  if (gate == GSA_GATE_LEARNED && !w_g) return GSA_ERR_INVALID_ARG;
+  if (no_sel && sel_idx_out) return GSA_ERR_INVALID_ARG;
   DeviceGuard dg(c->device);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   c->last_stream = st;
@@ -266,7 +273,8 @@ int gsa_forward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void* 
     a.tiles0 = a.tiles_total = a.tiles_per_split = attn_tc_tiles(d.R); a.n_split = 1;
     a.H = H; a.g = g; a.scale_log2 = scale * LOG2E;
     a.o32 = c->at<float>(c->L.ocomp); a.o_hs = rhs;
-    a.kc = d.kc; a.cand = c->at<int>(c->L.idx); a.cand_user = sel_idx_out;
+    a.kc = no_sel ? 0 : d.kc; a.cand = c->at<int>(c->L.idx); a.cand_user = sel_idx_out;
+    a.guide_only = cf.variant == GSA_VARIANT_NO_COMP_VALUE ? 1 : 0;
     a.rpf = d.rpf; a.n_fixed = cf.num_fixed_frames;
     for (int i = 0; i < cf.num_fixed_frames; ++i) a.fixed[i] = c->fixed[i];
     a.err = err;
@@ -284,9 +292,9 @@ int gsa_forward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void* 
     a.kc = d.kc; a.cand = c->at<int>(c->L.idx); a.cand_user = sel_idx_out;
     a.rpf = d.rpf; a.n_fixed = cf.num_fixed_frames;
     for (int i = 0; i < cf.num_fixed_frames; ++i) a.fixed[i] = c->fixed[i];
-    if (launch_attn_f32(a, true, st) != cudaSuccess) return GSA_ERR_CUDA;
+    if (launch_attn_f32(a, !no_sel, st) != cudaSuccess) return GSA_ERR_CUDA;
   }
-  prof.mark("comp_attn_topk");
+  prof.mark(no_sel ? "comp_attn" : cf.variant == GSA_VARIANT_NO_COMP_VALUE ? "comp_guide_topk" : "comp_attn_topk");
 
   // K3 selection (+ K4 upsample/gate/blend, fused for bf16)
   SelArgs sa;
@@ -299,8 +307,13 @@ int gsa_forward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void* 
   EpiArgs ea;
   ea.q_img = q_img; ea.o_sel = c->ws + c->L.osel; ea.o_comp = c->at<float>(c->L.ocomp);
   ea.w_g = w_g; ea.o_img = o_img; ea.H = H; ea.F = cf.num_frames; ea.R = d.R; ea.rpf = d.rpf;
-  ea.s = cf.pool_s; ea.g = g; ea.gate_mode = cf.gate_mode;
-  if (!d.fp32) {
+  ea.s = cf.pool_s; ea.g = g; ea.gate_mode = gate;
+  if (no_sel) {
+    // no selection branch: the epilogue only upsamples O'_comp (O_sel is never read)
+    ea.o_sel = nullptr;
+    if (launch_epilogue(ea, d.fp32, st) != cudaSuccess) return GSA_ERR_CUDA;
+    prof.mark("upsample");
+  } else if (!d.fp32) {
     // O_sel is written only when the caller asked to keep intermediates
     if (!(c->profiling & GSA_PROFILE_KEEP_OSEL)) sa.o_sel = nullptr;
     if (launch_sel_fused(sa, ea, st) != cudaSuccess) return GSA_ERR_CUDA;

@@ -31,7 +31,8 @@ struct AttnArgs {
   long long kv_hs[2];
   int n_k[2];
   int kmask[2];              // MaskMode per segment
-  int tiles0;                // 64-key tiles of segment 0
+  int guide_only;            // top-k only: S and the top-k, no P V and no output
+  int tiles0;                // 128-key tiles of segment 0
   int tiles_total;
   int tiles_per_split;
   int n_split;               // 1 = write final output, >1 = write partials

@@ -297,7 +297,8 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) sel_kernel_bf16(const SelArgs 
         if (qv) {
           const float2 gg = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gp[nt][rr]));
           const float g0 = gg.x, g1 = gg.y;
-          const float2 oc = __ldg(reinterpret_cast<const float2*>(cr + c));
+          // g = 0 (no compressed value) never reads O'_comp, which may not exist
+          const float2 oc = ep.gate_mode == 2 ? make_float2(0.f, 0.f) : __ldg(reinterpret_cast<const float2*>(cr + c));
           out0 = g0 * oc.x + (1.f - g0) * s0;
           out1 = g1 * oc.y + (1.f - g1) * s1;
         }
