@@ -144,6 +144,25 @@ __device__ __forceinline__ uint32_t pick64(const uint32_t* v, int e) {
   return sel_if(e & 1, t[1], t[0]);
 }
 
+// Two exponentials of the softmax with packed fp32x2 arithmetic (one FFMA2
+// for both arguments, one FADD2 for both running sums): half the FMA-pipe
+// issue slots of the scalar form, and exactly its roundings.
+__device__ __forceinline__ void exp2_pair(uint32_t s0, uint32_t s1, float sl2, float nmb, float& l0, float& l1,
+                                          float& p0, float& p1) {
+  float x0, x1;
+  asm("{\n .reg .b64 a, b, c, d;\n"
+      " mov.b64 a, {%2, %3};\n mov.b64 b, {%4, %4};\n mov.b64 c, {%5, %5};\n"
+      " fma.rn.f32x2 d, a, b, c;\n mov.b64 {%0, %1}, d;\n}\n"
+      : "=f"(x0), "=f"(x1)
+      : "r"(s0), "r"(s1), "f"(sl2), "f"(nmb));
+  p0 = ex2(x0);
+  p1 = ex2(x1);
+  asm("{\n .reg .b64 a, b;\n"
+      " mov.b64 a, {%0, %1};\n mov.b64 b, {%2, %3};\n add.rn.f32x2 a, a, b;\n mov.b64 {%0, %1}, a;\n}\n"
+      : "+f"(l0), "+f"(l1)
+      : "f"(p0), "f"(p1));
+}
+
 // max of 32 values with 4 independent chains
 __device__ __forceinline__ float max32(const uint32_t* v) {
   float m0 = __uint_as_float(v[0]), m1 = __uint_as_float(v[1]), m2 = __uint_as_float(v[2]),
@@ -444,10 +463,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float p0 = ex2(fmaf(__uint_as_float(v[32 * c + e]), sl2, -mb));
-            const float p1 = ex2(fmaf(__uint_as_float(v[32 * c + e + 1]), sl2, -mb));
-            l0 += p0;
-            l1 += p1;
+            float p0, p1;
+            exp2_pair(v[32 * c + e], v[32 * c + e + 1], sl2, -mb, l0, l1, p0, p1);
             pk[e >> 1] = pack_bf16(p0, p1);
           }
           tmem_st16(tP + 16 * c, pk);
@@ -526,10 +543,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           uint32_t pk[32];
 #pragma unroll
           for (int e = 0; e < 64; e += 2) {
-            const float p0 = ex2(fmaf(__uint_as_float(v[e]), sl2, -mb));
-            const float p1 = ex2(fmaf(__uint_as_float(v[e + 1]), sl2, -mb));
-            l0 += p0;
-            l1 += p1;
+            float p0, p1;
+            exp2_pair(v[e], v[e + 1], sl2, -mb, l0, l1, p0, p1);
             pk[e >> 1] = pack_bf16(p0, p1);
           }
           tmem_st32(tP + 32 * hf, pk);
