@@ -398,11 +398,9 @@ def run_b200(args, cfg, rank, world, local, dist):
         d2h = sum(t.numel() * t.element_size() for t in ho.values())
 
         def e2e_step():
-            for k in hx:
-                x[k].copy_(hx[k], non_blocking=True)
-            layer.forward(x, out=out)
-            for k in ho:
-                ho[k].copy_(out[k], non_blocking=True)
+            # gsa_forward_host: pinned host inputs in, pinned host outputs out, the
+            # copies overlapped with the layer chunk by chunk over the heads
+            layer.forward_host(hx, ho)
 
         e2e_step()
         torch.cuda.synchronize()

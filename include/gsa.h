@@ -131,6 +131,24 @@ GSA_API int gsa_forward(gsa_ctx *ctx,
                 const void *w_g, void *o_spec, void *o_img, int32_t *sel_idx_out,
                 void *stream);
 
+/* gsa_forward with HOST buffers: the same arguments and layouts, every tensor
+ * pointer (inputs, outputs, optional sel_idx_out) in host memory.  The heads
+ * are processed in up to four chunks: the host-to-device copies of chunk i+1
+ * and the device-to-host copies of chunk i-1 overlap the layer on chunk i
+ * (two extra streams of the context).  Asynchronous on `stream`: the outputs
+ * are in host memory once `stream` has completed; the inputs may be reused
+ * then too.  Overlap needs page-locked host memory (cudaHostAlloc or
+ * cudaHostRegister); pageable memory still gives correct results, with the
+ * copies serialised by the driver.  On first use the context allocates device
+ * copies of one call's inputs and outputs (GSA_ERR_OOM if that fails); they
+ * are freed by gsa_destroy.  The special-token split count is chosen per
+ * chunk, so o_spec may differ from gsa_forward's in the last bits. */
+GSA_API int gsa_forward_host(gsa_ctx *ctx,
+                             const void *q_spec, const void *k_spec, const void *v_spec,
+                             const void *q_img, const void *k_img, const void *v_img,
+                             const void *w_g, void *o_spec, void *o_img,
+                             int32_t *sel_idx_out, void *stream);
+
 /* Dense global attention over every token of the same shape (the comparison
  * baseline, "Full Attn." in the notes' latency table):
  *   q, k, v, o : [H][F*(num_special + pad_h*pad_w)][64], per frame the special

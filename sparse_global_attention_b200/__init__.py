@@ -24,7 +24,7 @@ GSA_PROFILE_TIMES, GSA_PROFILE_KEEP_OSEL = 1, 2
 EXPORTED = ("gsa_create", "gsa_workspace_bytes", "gsa_forward", "gsa_dense_forward",
             "gsa_get_intermediate", "gsa_set_profiling", "gsa_get_kernel_times",
             "gsa_get_status", "gsa_strerror", "gsa_destroy", "gsa_special_attention_noalloc",
-            "gsa_debug_expire_wait")
+            "gsa_debug_expire_wait", "gsa_forward_host")
 
 
 class gsa_config(ctypes.Structure):
@@ -240,6 +240,30 @@ class GSALayer:
                     x["w_g"].data_ptr(), out["o_spec"].data_ptr() if has_spec else 0,
                     out["o_img"].data_ptr(), 0 if sel_idx is None else sel_idx.data_ptr(), st)
         return out
+
+    def forward_host(self, hx, hout, sel_idx=None, stream=None):
+        """The layer on host tensors (gsa_forward_host): hx/hout hold CPU tensors
+        with the layouts of forward(); pinned memory lets the copies overlap the
+        compute.  Asynchronous on the stream like forward()."""
+        import torch
+        for k in ("q_img", "k_img", "v_img", "q_spec", "k_spec", "v_spec", "w_g"):
+            t = hx[k]
+            if t.is_cuda or not t.is_contiguous():
+                raise GSAError(f"{k} must be a contiguous host tensor")
+        st = stream if stream is not None else torch.cuda.current_stream().cuda_stream
+        has_spec = hx["q_spec"].numel() > 0
+        fn = load_library().gsa_forward_host
+        fn.argtypes = [ctypes.c_void_p] * 12
+        fn.restype = ctypes.c_int
+        _check(fn(self.ctx,
+                  hx["q_spec"].data_ptr() if has_spec else None,
+                  hx["k_spec"].data_ptr() if has_spec else None,
+                  hx["v_spec"].data_ptr() if has_spec else None,
+                  hx["q_img"].data_ptr(), hx["k_img"].data_ptr(), hx["v_img"].data_ptr(),
+                  hx["w_g"].data_ptr(), hout["o_spec"].data_ptr() if has_spec else None,
+                  hout["o_img"].data_ptr(), None if sel_idx is None else sel_idx.data_ptr(), st or None),
+               "gsa_forward_host")
+        return hout
 
     def dense(self, q, k, v, o=None, stream=None):
         import torch

@@ -13,6 +13,7 @@ namespace {
 
 constexpr size_t ALIGN = 256;
 constexpr int MAX_EVENTS = 16;
+constexpr int MAX_CHUNKS = 8;          // head chunks of the host-buffer pipeline
 
 size_t align_up(size_t x) { return (x + ALIGN - 1) / ALIGN * ALIGN; }
 
@@ -110,6 +111,12 @@ struct gsa_ctx {
   cudaEvent_t ev[MAX_EVENTS];
   const char* ev_names[MAX_EVENTS];
   int n_ev;
+  // host-buffer path (gsa_forward_host): device copies of one call's inputs and
+  // outputs, copy streams and per-chunk events, created on first use
+  uint8_t* stage;
+  size_t stage_bytes;
+  cudaStream_t s_in, s_out;
+  cudaEvent_t ev_start, ev_in[MAX_CHUNKS], ev_comp[MAX_CHUNKS], ev_out;
   template <typename T>
   T* at(size_t off) const { return off == SIZE_MAX ? nullptr : reinterpret_cast<T*>(ws + off); }
 };
@@ -142,12 +149,15 @@ Grid grid_of(const gsa_config& c) {
 struct Prof {
   gsa_ctx* ctx;
   cudaStream_t st;
-  Prof(gsa_ctx* c, cudaStream_t s) : ctx(c), st(s) {
+  bool on;
+  Prof(gsa_ctx* c, cudaStream_t s, bool timing = true)
+      : ctx(c), st(s), on(timing && (c->profiling & GSA_PROFILE_TIMES)) {
+    if (!on) return;
     ctx->n_ev = 0;
-    if (ctx->profiling & GSA_PROFILE_TIMES) cudaEventRecord(ctx->ev[ctx->n_ev++], st);
+    cudaEventRecord(ctx->ev[ctx->n_ev++], st);
   }
   void mark(const char* name) {
-    if ((ctx->profiling & GSA_PROFILE_TIMES) && ctx->n_ev < MAX_EVENTS) {
+    if (on && ctx->n_ev < MAX_EVENTS) {
       ctx->ev_names[ctx->n_ev - 1] = name;
       cudaEventRecord(ctx->ev[ctx->n_ev++], st);
     }
@@ -214,18 +224,35 @@ int gsa_create(const gsa_config* cfg, gsa_ctx** out) {
 void gsa_destroy(gsa_ctx* c) {
   if (!c) return;
   DeviceGuard dg(c->device);
+  if (c->stage) {
+    cudaFree(c->stage);
+    cudaStreamDestroy(c->s_in);
+    cudaStreamDestroy(c->s_out);
+    cudaEventDestroy(c->ev_start);
+    cudaEventDestroy(c->ev_out);
+    for (int i = 0; i < MAX_CHUNKS; ++i) {
+      cudaEventDestroy(c->ev_in[i]);
+      cudaEventDestroy(c->ev_comp[i]);
+    }
+  }
   for (int i = 0; i < MAX_EVENTS; ++i) cudaEventDestroy(c->ev[i]);
   cudaFree(c->ws);
   delete c;
 }
 
-int gsa_forward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void* v_spec,
-                const void* q_img, const void* k_img, const void* v_img, const void* w_g,
-                void* o_spec, void* o_img, int32_t* sel_idx_out, void* stream) {
-  if (!c || !q_img || !k_img || !v_img || !o_img) return GSA_ERR_INVALID_ARG;
+}  // extern "C"
+
+namespace {
+
+// The layer for heads [h0, h0 + nh) of the context: every tensor argument
+// points at head 0 of its full [H]... array; workspace rows of those heads are
+// used, the special-token partials from their start (capacity n_split * H rows
+// per query, split count chosen for nh heads within it).
+int forward_heads(gsa_ctx* c, int h0, int nh, const void* q_spec, const void* k_spec, const void* v_spec,
+                  const void* q_img, const void* k_img, const void* v_img, const void* w_g,
+                  void* o_spec, void* o_img, int32_t* sel_idx_out, cudaStream_t st, bool timing) {
   const gsa_config& cf = c->cfg;
   const Derived& d = c->d;
-  if (cf.num_special > 0 && (!q_spec || !k_spec || !v_spec || !o_spec)) return GSA_ERR_INVALID_ARG;
   // the ablation variants fix the blend: no compressed value -> O_sel, no selection -> O_comp
   const int gate = cf.variant == GSA_VARIANT_NO_COMP_VALUE ? GSA_GATE_SEL_ONLY
                    : cf.variant == GSA_VARIANT_NO_SELECTION ? GSA_GATE_COMP_ONLY
@@ -233,25 +260,52 @@ int gsa_forward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void* 
   const bool no_sel = cf.variant == GSA_VARIANT_NO_SELECTION;
   if (gate == GSA_GATE_LEARNED && !w_g) return GSA_ERR_INVALID_ARG;
   if (no_sel && sel_idx_out) return GSA_ERR_INVALID_ARG;
-  DeviceGuard dg(c->device);
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  c->last_stream = st;
-  const int H = cf.num_heads;
+  const int H = nh;
+  // per-head strides in bytes, and the views of heads [h0, h0 + nh)
+  const size_t es = d.esize;
+  const size_t img_b = static_cast<size_t>(d.img_per_head) * D * es;
+  const size_t spec_b = static_cast<size_t>(d.spec_per_head) * D * es;
+  const size_t rrow = static_cast<size_t>(d.R) * D;
+  auto off = [&](const void* p, size_t per_head) -> const void* {
+    return p ? static_cast<const uint8_t*>(p) + static_cast<size_t>(h0) * per_head : nullptr;
+  };
+  auto offm = [&](void* p, size_t per_head) -> void* {
+    return p ? static_cast<uint8_t*>(p) + static_cast<size_t>(h0) * per_head : nullptr;
+  };
+  auto ws = [&](size_t o, size_t per_head) -> uint8_t* {
+    return o == SIZE_MAX ? nullptr : c->ws + o + static_cast<size_t>(h0) * per_head;
+  };
+  q_img = off(q_img, img_b); k_img = off(k_img, img_b); v_img = off(v_img, img_b);
+  q_spec = off(q_spec, spec_b); k_spec = off(k_spec, spec_b); v_spec = off(v_spec, spec_b);
+  w_g = off(w_g, static_cast<size_t>(D) * D * es);
+  o_img = offm(o_img, img_b); o_spec = offm(o_spec, spec_b);
+  if (sel_idx_out) sel_idx_out += static_cast<size_t>(h0) * d.R * cf.topk;
+  __nv_bfloat16* comp16[3];
+  __nv_bfloat16* complo[2];
+  float* comp32[3];
+  for (int i = 0; i < 3; ++i) {
+    comp16[i] = reinterpret_cast<__nv_bfloat16*>(ws(c->L.comp16[i], rrow * 2));
+    comp32[i] = reinterpret_cast<float*>(ws(c->L.comp32[i], rrow * 4));
+  }
+  for (int i = 0; i < 2; ++i) complo[i] = reinterpret_cast<__nv_bfloat16*>(ws(c->L.complo[i], rrow * 2));
+  float* ocomp = reinterpret_cast<float*>(ws(c->L.ocomp, rrow * 4));
+  int* idx = reinterpret_cast<int*>(ws(c->L.idx, static_cast<size_t>(d.R) * cf.topk * 4));
+  uint8_t* osel = ws(c->L.osel, img_b);
   const Grid g = grid_of(cf);
   const float scale = scale_of(cf);
   int* err = c->at<int>(c->L.err);
   if (!k_spec) k_spec = k_img;   // never dereferenced without special/fixed tokens
   if (!v_spec) v_spec = v_img;
   if (!w_g) w_g = q_img;         // never read when the gate is forced
-  Prof prof(c, st);
+  Prof prof(c, st, timing);
 
   // K1 pool
   PoolArgs pa;
   pa.src[0] = q_img; pa.src[1] = k_img; pa.src[2] = v_img;
   for (int i = 0; i < 3; ++i) {
-    pa.out16[i] = c->at<__nv_bfloat16>(c->L.comp16[i]);
-    pa.outlo[i] = i < 2 ? c->at<__nv_bfloat16>(c->L.complo[i]) : nullptr;
-    pa.out32[i] = c->at<float>(c->L.comp32[i]);
+    pa.out16[i] = comp16[i];
+    pa.outlo[i] = i < 2 ? complo[i] : nullptr;
+    pa.out32[i] = comp32[i];
   }
   pa.H = H; pa.F = cf.num_frames; pa.Hp = cf.pad_h; pa.Wp = cf.pad_w;
   pa.Hv = cf.grid_h; pa.Wv = cf.grid_w; pa.s = cf.pool_s;
@@ -263,17 +317,17 @@ int gsa_forward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void* 
   if (!d.fp32) {
     AttnArgs a;
     memset(&a, 0, sizeof(a));
-    a.q = c->at<__nv_bfloat16>(c->L.comp16[0]); a.q_hs = rhs; a.n_q = d.R; a.q_mask = MASK_NONE;
-    a.q_lo = c->at<__nv_bfloat16>(c->L.complo[0]); a.k_lo = c->at<__nv_bfloat16>(c->L.complo[1]);
+    a.q = comp16[0]; a.q_hs = rhs; a.n_q = d.R; a.q_mask = MASK_NONE;
+    a.q_lo = complo[0]; a.k_lo = complo[1];
     a.nseg = 1;
-    a.k[0] = a.k[1] = c->at<__nv_bfloat16>(c->L.comp16[1]);
-    a.v[0] = a.v[1] = c->at<__nv_bfloat16>(c->L.comp16[2]);
+    a.k[0] = a.k[1] = comp16[1];
+    a.v[0] = a.v[1] = comp16[2];
     a.kv_hs[0] = a.kv_hs[1] = rhs; a.n_k[0] = a.n_k[1] = d.R;
     a.kmask[0] = a.kmask[1] = MASK_NONE;
     a.tiles0 = a.tiles_total = a.tiles_per_split = attn_tc_tiles(d.R); a.n_split = 1;
     a.H = H; a.g = g; a.scale_log2 = scale * LOG2E;
-    a.o32 = c->at<float>(c->L.ocomp); a.o_hs = rhs;
-    a.kc = no_sel ? 0 : d.kc; a.cand = c->at<int>(c->L.idx); a.cand_user = sel_idx_out;
+    a.o32 = ocomp; a.o_hs = rhs;
+    a.kc = no_sel ? 0 : d.kc; a.cand = idx; a.cand_user = sel_idx_out;
     a.guide_only = cf.variant == GSA_VARIANT_NO_COMP_VALUE ? 1 : 0;
     a.rpf = d.rpf; a.n_fixed = cf.num_fixed_frames;
     for (int i = 0; i < cf.num_fixed_frames; ++i) a.fixed[i] = c->fixed[i];
@@ -282,14 +336,14 @@ int gsa_forward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void* 
   } else {
     AttnF32Args a;
     memset(&a, 0, sizeof(a));
-    a.q = c->at<float>(c->L.comp32[0]); a.q_hs = rhs; a.n_q = d.R; a.q_mask = MASK_NONE;
+    a.q = comp32[0]; a.q_hs = rhs; a.n_q = d.R; a.q_mask = MASK_NONE;
     a.nseg = 1;
-    a.k[0] = a.k[1] = c->at<float>(c->L.comp32[1]);
-    a.v[0] = a.v[1] = c->at<float>(c->L.comp32[2]);
+    a.k[0] = a.k[1] = comp32[1];
+    a.v[0] = a.v[1] = comp32[2];
     a.kv_hs[0] = a.kv_hs[1] = rhs; a.n_k[0] = a.n_k[1] = d.R;
     a.H = H; a.g = g; a.scale = scale;
-    a.o = c->at<float>(c->L.ocomp); a.o_hs = rhs;
-    a.kc = d.kc; a.cand = c->at<int>(c->L.idx); a.cand_user = sel_idx_out;
+    a.o = ocomp; a.o_hs = rhs;
+    a.kc = d.kc; a.cand = idx; a.cand_user = sel_idx_out;
     a.rpf = d.rpf; a.n_fixed = cf.num_fixed_frames;
     for (int i = 0; i < cf.num_fixed_frames; ++i) a.fixed[i] = c->fixed[i];
     if (launch_attn_f32(a, !no_sel, st) != cudaSuccess) return GSA_ERR_CUDA;
@@ -299,13 +353,13 @@ int gsa_forward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void* 
   // K3 selection (+ K4 upsample/gate/blend, fused for bf16)
   SelArgs sa;
   sa.q_img = q_img; sa.k_img = k_img; sa.v_img = v_img; sa.k_spec = k_spec; sa.v_spec = v_spec;
-  sa.idx = c->at<int>(c->L.idx); sa.o_sel = c->ws + c->L.osel;
+  sa.idx = idx; sa.o_sel = osel;
   sa.H = H; sa.F = cf.num_frames; sa.R = d.R; sa.rpf = d.rpf; sa.topk = cf.topk; sa.s = cf.pool_s;
   sa.g = g; sa.scale_log2 = scale * LOG2E; sa.n_fixed = cf.num_fixed_frames;
   for (int i = 0; i < cf.num_fixed_frames; ++i) sa.fixed[i] = c->fixed[i];
   sa.err = err;
   EpiArgs ea;
-  ea.q_img = q_img; ea.o_sel = c->ws + c->L.osel; ea.o_comp = c->at<float>(c->L.ocomp);
+  ea.q_img = q_img; ea.o_sel = osel; ea.o_comp = ocomp;
   ea.w_g = w_g; ea.o_img = o_img; ea.H = H; ea.F = cf.num_frames; ea.R = d.R; ea.rpf = d.rpf;
   ea.s = cf.pool_s; ea.g = g; ea.gate_mode = gate;
   if (no_sel) {
@@ -325,7 +379,17 @@ int gsa_forward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void* 
     prof.mark("epilogue");
   }
 
-  // K5 special tokens over every token
+  // K5 special tokens over every token; the split count fills the GPU for nh
+  // heads, within the partials' capacity (d.spec_split splits of all H heads)
+  int tps = d.spec_tps, nsplit = d.spec_split;
+  if (nh != cf.num_heads && cf.num_special > 0) {
+    attn_tc_split(nh, d.spec_per_head, d.spec_tiles_total, &tps, &nsplit);
+    const int cap = static_cast<int>((static_cast<long long>(d.spec_split) * cf.num_heads) / nh);
+    if (nsplit > cap) {
+      tps = (d.spec_tiles_total + cap - 1) / cap;
+      nsplit = (d.spec_tiles_total + tps - 1) / tps;
+    }
+  }
   if (cf.num_special > 0) {
     const long long shs = d.spec_per_head * D;
     const long long ihs = d.img_per_head * D;
@@ -343,16 +407,16 @@ int gsa_forward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void* 
       a.kv_hs[1] = ihs; a.n_k[1] = static_cast<int>(d.img_per_head);
       a.kmask[1] = d.pads ? MASK_IMG : MASK_NONE;
       a.tiles0 = d.spec_tiles0; a.tiles_total = d.spec_tiles_total;
-      a.tiles_per_split = d.spec_tps; a.n_split = d.spec_split;
+      a.tiles_per_split = tps; a.n_split = nsplit;
       a.H = H; a.g = g; a.scale_log2 = scale * LOG2E;
       a.o16 = reinterpret_cast<__nv_bfloat16*>(o_spec); a.o_hs = shs;
       a.part_o = c->at<float>(c->L.part_o); a.part_ml = c->at<float>(c->L.part_ml);
       a.err = err;
       if (launch_attn_tc(a, st) != cudaSuccess) return GSA_ERR_CUDA;
       prof.mark("special");
-      if (d.spec_split > 1) {
+      if (nsplit > 1) {
         MergeArgs m;
-        m.part_o = a.part_o; m.part_ml = a.part_ml; m.n_split = d.spec_split; m.H = H;
+        m.part_o = a.part_o; m.part_ml = a.part_ml; m.n_split = nsplit; m.H = H;
         m.n_q = a.n_q; m.scale_log2 = a.scale_log2; m.o16 = a.o16; m.o32 = nullptr; m.o_hs = shs;
         if (launch_merge(m, st) != cudaSuccess) return GSA_ERR_CUDA;
         prof.mark("special_merge");
@@ -374,6 +438,115 @@ int gsa_forward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void* 
       prof.mark("special");
     }
   }
+  return GSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gsa_forward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void* v_spec,
+                const void* q_img, const void* k_img, const void* v_img, const void* w_g,
+                void* o_spec, void* o_img, int32_t* sel_idx_out, void* stream) {
+  if (!c || !q_img || !k_img || !v_img || !o_img) return GSA_ERR_INVALID_ARG;
+  const gsa_config& cf = c->cfg;
+  if (cf.num_special > 0 && (!q_spec || !k_spec || !v_spec || !o_spec)) return GSA_ERR_INVALID_ARG;
+  const int gate = cf.variant == GSA_VARIANT_NO_COMP_VALUE ? GSA_GATE_SEL_ONLY
+                   : cf.variant == GSA_VARIANT_NO_SELECTION ? GSA_GATE_COMP_ONLY
+                                                            : cf.gate_mode;
+  if (gate == GSA_GATE_LEARNED && !w_g) return GSA_ERR_INVALID_ARG;
+  if (cf.variant == GSA_VARIANT_NO_SELECTION && sel_idx_out) return GSA_ERR_INVALID_ARG;
+  DeviceGuard dg(c->device);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  c->last_stream = st;
+  return forward_heads(c, 0, cf.num_heads, q_spec, k_spec, v_spec, q_img, k_img, v_img, w_g, o_spec, o_img,
+                       sel_idx_out, st, true);
+}
+
+int gsa_forward_host(gsa_ctx* c, const void* q_spec, const void* k_spec, const void* v_spec,
+                     const void* q_img, const void* k_img, const void* v_img, const void* w_g,
+                     void* o_spec, void* o_img, int32_t* sel_idx_out, void* stream) {
+  if (!c || !q_img || !k_img || !v_img || !o_img) return GSA_ERR_INVALID_ARG;
+  const gsa_config& cf = c->cfg;
+  const Derived& d = c->d;
+  const bool spec = cf.num_special > 0;
+  if (spec && (!q_spec || !k_spec || !v_spec || !o_spec)) return GSA_ERR_INVALID_ARG;
+  const int gate = cf.variant == GSA_VARIANT_NO_COMP_VALUE ? GSA_GATE_SEL_ONLY
+                   : cf.variant == GSA_VARIANT_NO_SELECTION ? GSA_GATE_COMP_ONLY
+                                                            : cf.gate_mode;
+  if (gate == GSA_GATE_LEARNED && !w_g) return GSA_ERR_INVALID_ARG;
+  if (cf.variant == GSA_VARIANT_NO_SELECTION && sel_idx_out) return GSA_ERR_INVALID_ARG;
+  DeviceGuard dg(c->device);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int H = cf.num_heads;
+  const size_t es = d.esize;
+  const size_t img_b = static_cast<size_t>(d.img_per_head) * D * es;
+  const size_t spec_b = static_cast<size_t>(d.spec_per_head) * D * es;
+  const size_t wg_b = static_cast<size_t>(D) * D * es;
+  const size_t idx_b = static_cast<size_t>(d.R) * cf.topk * 4;
+  const bool wg = gate == GSA_GATE_LEARNED;
+  // device copies: q/k/v_img, q/k/v_spec, w_g, o_img, o_spec, idx ([H]... each)
+  size_t offs[10], tot = 0;
+  const size_t per[10] = {img_b, img_b, img_b, spec_b, spec_b, spec_b, wg_b, img_b, spec_b, idx_b};
+  for (int i = 0; i < 10; ++i) {
+    offs[i] = tot;
+    tot = align_up(tot + per[i] * H);
+  }
+  if (!c->stage) {
+    if (cudaMalloc(&c->stage, tot) != cudaSuccess) {
+      c->stage = nullptr;
+      return GSA_ERR_OOM;
+    }
+    c->stage_bytes = tot;
+    if (cudaStreamCreateWithFlags(&c->s_in, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&c->s_out, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&c->ev_start, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&c->ev_out, cudaEventDisableTiming) != cudaSuccess)
+      return GSA_ERR_CUDA;
+    for (int i = 0; i < MAX_CHUNKS; ++i)
+      if (cudaEventCreateWithFlags(&c->ev_in[i], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&c->ev_comp[i], cudaEventDisableTiming) != cudaSuccess)
+        return GSA_ERR_CUDA;
+  }
+  uint8_t* dp[10];
+  for (int i = 0; i < 10; ++i) dp[i] = c->stage + offs[i];
+  const void* hin[7] = {q_img, k_img, v_img, q_spec, k_spec, v_spec, w_g};
+  // chunks of heads: copies of chunk i+1 in overlap the layer on chunk i, whose
+  // outputs go back while chunk i+1 computes
+  const int nchunk = H < 4 ? H : 4;
+  const int hpc = (H + nchunk - 1) / nchunk;
+  if (cudaEventRecord(c->ev_start, st) != cudaSuccess) return GSA_ERR_CUDA;
+  if (cudaStreamWaitEvent(c->s_in, c->ev_start, 0) != cudaSuccess) return GSA_ERR_CUDA;
+  int k = 0;
+  for (int h0 = 0; h0 < H; h0 += hpc, ++k) {
+    const int nh = (h0 + hpc <= H) ? hpc : H - h0;
+    for (int i = 0; i < 7; ++i) {
+      if ((i >= 3 && i < 6 && !spec) || (i == 6 && !wg) || per[i] == 0) continue;
+      if (cudaMemcpyAsync(dp[i] + h0 * per[i], static_cast<const uint8_t*>(hin[i]) + h0 * per[i], nh * per[i],
+                          cudaMemcpyHostToDevice, c->s_in) != cudaSuccess)
+        return GSA_ERR_CUDA;
+    }
+    if (cudaEventRecord(c->ev_in[k], c->s_in) != cudaSuccess) return GSA_ERR_CUDA;
+    if (cudaStreamWaitEvent(st, c->ev_in[k], 0) != cudaSuccess) return GSA_ERR_CUDA;
+    const int rc = forward_heads(c, h0, nh, spec ? dp[3] : nullptr, spec ? dp[4] : nullptr, spec ? dp[5] : nullptr,
+                                 dp[0], dp[1], dp[2], wg ? dp[6] : nullptr, spec ? dp[8] : nullptr, dp[7],
+                                 sel_idx_out ? reinterpret_cast<int32_t*>(dp[9]) : nullptr, st, false);
+    if (rc != GSA_OK) return rc;
+    if (cudaEventRecord(c->ev_comp[k], st) != cudaSuccess) return GSA_ERR_CUDA;
+    if (cudaStreamWaitEvent(c->s_out, c->ev_comp[k], 0) != cudaSuccess) return GSA_ERR_CUDA;
+    void* hout[3] = {o_img, spec ? o_spec : nullptr, sel_idx_out};
+    const int src[3] = {7, 8, 9};
+    for (int i = 0; i < 3; ++i) {
+      if (!hout[i] || per[src[i]] == 0) continue;
+      if (cudaMemcpyAsync(static_cast<uint8_t*>(hout[i]) + h0 * per[src[i]], dp[src[i]] + h0 * per[src[i]],
+                          nh * per[src[i]], cudaMemcpyDeviceToHost, c->s_out) != cudaSuccess)
+        return GSA_ERR_CUDA;
+    }
+  }
+  // the caller's stream completes when the last output has reached the host
+  if (cudaEventRecord(c->ev_out, c->s_out) != cudaSuccess) return GSA_ERR_CUDA;
+  if (cudaStreamWaitEvent(st, c->ev_out, 0) != cudaSuccess) return GSA_ERR_CUDA;
+  c->last_stream = st;
   return GSA_OK;
 }
 
