@@ -513,7 +513,7 @@ int gsa_forward_host(gsa_ctx* c, const void* q_spec, const void* k_spec, const v
   const void* hin[7] = {q_img, k_img, v_img, q_spec, k_spec, v_spec, w_g};
   // chunks of heads: copies of chunk i+1 in overlap the layer on chunk i, whose
   // outputs go back while chunk i+1 computes
-  const int nchunk = H < 4 ? H : 4;
+  const int nchunk = H < MAX_CHUNKS ? H : MAX_CHUNKS;
   const int hpc = (H + nchunk - 1) / nchunk;
   if (cudaEventRecord(c->ev_start, st) != cudaSuccess) return GSA_ERR_CUDA;
   if (cudaStreamWaitEvent(c->s_in, c->ev_start, 0) != cudaSuccess) return GSA_ERR_CUDA;
