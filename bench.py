@@ -441,9 +441,19 @@ def run_b200(args, cfg, rank, world, local, dist):
     if args.ablations:
         ablations = {}
         specs = [("no_comp_value", dict(variant="no_comp_value")), ("no_selection", dict(variant="no_selection")),
-                 ("top8", dict(topk=8)), ("top16", dict(topk=16)), ("top64", dict(topk=64))]
+                 ("top8", dict(topk=8)), ("top16", dict(topk=16)), ("top64", dict(topk=64)), ("windows8x8", None)]
         for name, kw in specs:
-            lay = gsa.GSALayer.from_workload(cfg, **kw)
+            if kw is None:
+                # 8x8 windows: the grid padded to a multiple of 8, inputs drawn for that layout
+                pad = lambda n: (n + 7) // 8 * 8
+                wcfg = cfg.with_(pool_s=8, pad_h=pad(cfg.grid_h), pad_w=pad(cfg.grid_w))
+                del x, out
+                torch.cuda.empty_cache()
+                x = make_inputs(wcfg, seed=rank, device=dev)
+                out = {"o_img": torch.empty_like(x["q_img"]), "o_spec": torch.empty_like(x["q_spec"])}
+                lay = gsa.GSALayer.from_workload(wcfg)
+            else:
+                lay = gsa.GSALayer.from_workload(cfg, **kw)
             for _ in range(2):
                 lay.forward(x, out=out)
             torch.cuda.synchronize()

@@ -92,7 +92,7 @@ typedef struct {
                               camera tokens removed, pi^3 adaptation)             */
     int num_heads;         /* H >= 1                                              */
     int head_dim;          /* must be 64                                          */
-    int pool_s;            /* s in {1, 2, 4, 8} (bf16 path: {1, 2, 4})            */
+    int pool_s;            /* s in {1, 2, 4, 8}                                   */
     int topk;              /* regions per compressed query, 1..min(64, candidates) */
     int dtype;             /* GSA_BF16 or GSA_FP32                                */
     const int *fixed_frames; /* VGGT fixed global context frames (copied at

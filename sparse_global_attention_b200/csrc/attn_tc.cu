@@ -107,15 +107,44 @@ __device__ __forceinline__ int tile_seg(const AttnArgs& a, int tt, long long& kb
 }
 
 
-// validity bits of 32 consecutive keys starting at key0 (bit e = key0 + e)
+// validity bits of 32 consecutive keys starting at key0 (bit e = key0 + e).
+// A frame is `lead` always-valid keys (its special tokens, dense layout only)
+// and then Hp rows of Wp slots whose first Wv slots of the first Hv rows are
+// valid; the chunk is walked run by run (a handful of runs for 32 keys).
 __device__ __noinline__ uint32_t chunk_valid(int km, Grid g, int nk, long long key0) {
   const long long lim = nk - key0;
-  uint32_t m = lim >= 32 ? ~0u : (lim <= 0 ? 0u : ((1u << lim) - 1u));
-  if (km != MASK_NONE) {
-    for (int e = 0; e < 32; ++e)
-      if (((m >> e) & 1u) && !key_valid(km, g, key0 + e)) m &= ~(1u << e);
+  const uint32_t m = lim >= 32 ? ~0u : (lim <= 0 ? 0u : ((1u << lim) - 1u));
+  if (km == MASK_NONE || m == 0u) return m;
+  const int lead = km == MASK_DENSE ? g.ns : 0;
+  const int per = lead + g.Hp * g.Wp;
+  int o = static_cast<int>(key0 % per);
+  uint32_t v = 0;
+  for (int e = 0; e < 32;) {
+    int run;
+    bool ok;
+    if (o < lead) {
+      run = lead - o;
+      ok = true;
+    } else {
+      const int q = o - lead, y = q / g.Wp, x = q - y * g.Wp;
+      if (y >= g.Hv) {
+        run = per - o;                          // pad rows up to the end of the frame
+        ok = false;
+      } else if (x < g.Wv) {
+        run = g.Wv - x;
+        ok = true;
+      } else {
+        run = g.Wp - x;
+        ok = false;
+      }
+    }
+    const int n = min(run, 32 - e);
+    if (ok) v |= (n >= 32 ? ~0u : ((1u << n) - 1u)) << e;
+    e += n;
+    o += n;
+    if (o >= per) o -= per;
   }
-  return m;
+  return m & v;
 }
 
 // c ? a : b through an explicit selp, so that chains of these over a
@@ -260,7 +289,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const Bars bars{sbase + L::BAR, L::NST};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sgen + L::TMEM_SLOT);
 
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
   const int h = blockIdx.z, split = blockIdx.y;
   const int row0 = blockIdx.x * (2 * TBM);
   const int t_begin = split * a.tiles_per_split;

@@ -40,7 +40,6 @@ int validate(const gsa_config* c, Derived* d) {
   if (c->head_dim != 64) return GSA_ERR_SHAPE;
   const int s = c->pool_s;
   if (s != 1 && s != 2 && s != 4 && s != 8) return GSA_ERR_UNSUPPORTED;
-  if (c->dtype == GSA_BF16 && s == 8) return GSA_ERR_UNSUPPORTED;
   if (c->pad_h < c->grid_h || c->pad_w < c->grid_w) return GSA_ERR_SHAPE;
   if (c->pad_h % s || c->pad_w % s) return GSA_ERR_SHAPE;
   // every region needs a valid token: the last region row/col must reach the grid

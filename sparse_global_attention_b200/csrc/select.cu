@@ -9,7 +9,8 @@
 // frame and of the frames sampled every 100 frames.
 //
 // bf16 path (with the K4 epilogue fused in: O_img is written directly): one
-// warp per window (s*s <= 16 queries fill one m16 MMA tile);
+// warp per window (s*s <= 16 queries fill one m16 MMA tile; s = 8 takes four
+// warps per window, one per 16 queries);
 // 4 windows per CTA, neighbours in raster order so their overlapping region
 // choices meet in L2.  Each warp gathers its keys 32 at a time (the tokens of
 // the selected regions, then the fixed context) into its own double-buffered
@@ -95,7 +96,21 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) sel_kernel_bf16(const SelArgs 
   int2* sReg = reinterpret_cast<int2*>(wbase + 16 * 128 + 4 * SEL_TILE);
   uint8_t* sValid = reinterpret_cast<uint8_t*>(sReg + KC_MAX);
 
-  const long long win = static_cast<long long>(blockIdx.x) * SEL_WARPS + warp;
+  // RB row blocks of 16 queries per window.  s = 8: the CTA's four warps take
+  // one window, 16 queries each; they gather its keys together into the first
+  // warp's stages (8 keys per warp and block) and synchronise per block.
+  constexpr int RB = (S * S + 15) / 16;
+  constexpr bool SH = RB > 1;
+  static_assert(!SH || RB == SEL_WARPS, "one window per CTA");
+  const uint32_t sKVs = SH ? smem_u32(smem) + 16 * 128 : sKV;
+  uint8_t* sValidS = SH ? reinterpret_cast<uint8_t*>(reinterpret_cast<int2*>(smem + 16 * 128 + 4 * SEL_TILE) + KC_MAX)
+                        : sValid;
+  auto stage_sync = [&]() {
+    if constexpr (SH) __syncthreads(); else __syncwarp();
+  };
+  const long long wq = static_cast<long long>(blockIdx.x) * SEL_WARPS + warp;
+  const long long win = wq / RB;
+  const int rb = static_cast<int>(wq - win * RB);
   if (win >= static_cast<long long>(a.H) * a.R) return;      // warp-uniform
   const int h = static_cast<int>(win / a.R);
   const int r = static_cast<int>(win - static_cast<long long>(h) * a.R);
@@ -126,8 +141,9 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) sel_kernel_bf16(const SelArgs 
   for (int it = 0; it < 4; ++it) {
     const int e = lane + 32 * it;
     const int row = e >> 3, c = e & 7;
-    const int y = wi * S + row / S, x = wj * S + row % S;
-    const bool ok = row < S * S && y < a.g.Hv && x < a.g.Wv;
+    const int qr = 16 * rb + row;                  // query of the window
+    const int y = wi * S + qr / S, x = wj * S + qr % S;
+    const bool ok = qr < S * S && y < a.g.Hv && x < a.g.Wv;
     const long long tok = ok ? (static_cast<long long>(f) * a.g.Hp + y) * a.g.Wp + x : 0;
     cp_async16(sQ + swz(row, c), qh + tok * D + c * 8, ok ? 16 : 0);
   }
@@ -139,12 +155,12 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) sel_kernel_bf16(const SelArgs 
   const int nblk = (nkeys + SEL_BN - 1) / SEL_BN;
 
   auto issue = [&](int blk, int st) {
-    const uint32_t sK = sKV + st * 2 * SEL_TILE;
+    const uint32_t sK = sKVs + st * 2 * SEL_TILE;
     const uint32_t sV = sK + SEL_TILE;
 #pragma unroll
-    for (int it = 0; it < 8; ++it) {
+    for (int it = 0; it < (SH ? 2 : 8); ++it) {
       const int e = lane + 32 * it;
-      const int key = e >> 3, c = e & 7;
+      const int key = (SH ? 8 * warp : 0) + (e >> 3), c = e & 7;
       long long off;
       bool spec;
       const bool ok = key_src<S>(a, sReg, blk * SEL_BN + key, nk_dyn, nkeys, off, spec);
@@ -152,14 +168,14 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) sel_kernel_bf16(const SelArgs 
       const __nv_bfloat16* vp = (spec ? vsh : vh) + off * D + c * 8;
       cp_async16(sK + swz(key, c), ok ? kp : kh, ok ? 16 : 0);
       cp_async16(sV + swz(key, c), ok ? vp : vh, ok ? 16 : 0);
-      if (c == 0) sValid[st * SEL_BN + key] = ok ? 1 : 0;
+      if (c == 0) sValidS[st * SEL_BN + key] = ok ? 1 : 0;
     }
   };
 
   issue(0, 0);
   cp_async_commit();
   cp_async_wait<1>();
-  __syncwarp();
+  __syncwarp();                                   // this warp's Q
   uint32_t qf[4][4];
 #pragma unroll
   for (int ks = 0; ks < 4; ++ks)
@@ -200,12 +216,12 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) sel_kernel_bf16(const SelArgs 
 
   for (int blk = 0; blk < nblk; ++blk) {
     const int st = blk & 1;
-    __syncwarp();
+    stage_sync();                                 // every reader is done with stage st^1
     if (blk + 1 < nblk) issue(blk + 1, st ^ 1);
     cp_async_commit();
     cp_async_wait<1>();
-    __syncwarp();
-    const uint32_t sK = sKV + st * 2 * SEL_TILE;
+    stage_sync();                                 // every writer's part of stage st has landed
+    const uint32_t sK = sKVs + st * 2 * SEL_TILE;
     const uint32_t sV = sK + SEL_TILE;
 
     float s[4][4];
@@ -224,7 +240,7 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) sel_kernel_bf16(const SelArgs 
     for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
       for (int e = 0; e < 2; ++e)
-        if (!sValid[st * SEL_BN + 8 * nt + 2 * t + e]) {
+        if (!sValidS[st * SEL_BN + 8 * nt + 2 * t + e]) {
           s[nt][e] = -INFINITY;
           s[nt][2 + e] = -INFINITY;
         }
@@ -281,9 +297,9 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) sel_kernel_bf16(const SelArgs 
   for (int rr = 0; rr < 2; ++rr) {
     l[rr] += __shfl_xor_sync(0xffffffffu, l[rr], 1);
     l[rr] += __shfl_xor_sync(0xffffffffu, l[rr], 2);
-    const int row = g + 8 * rr;
-    if (row >= S * S) continue;
-    const int y = wi * S + row / S, x = wj * S + row % S;
+    const int qr = 16 * rb + g + 8 * rr;           // query of the window
+    if (qr >= S * S) continue;
+    const int y = wi * S + qr / S, x = wj * S + qr % S;
     const bool qv = y < a.g.Hv && x < a.g.Wv;
     const float inv = (qv && l[rr] > 0.f) ? 1.f / l[rr] : 0.f;
     const long long tok = (static_cast<long long>(f) * a.g.Hp + y) * a.g.Wp + x;
@@ -381,7 +397,7 @@ cudaError_t launch_sel_s(const SelArgs& a, bool fp32, cudaStream_t st) {
     const int sm = SEL_WARPS * SEL_WARP_SMEM;
     cudaError_t e = cudaFuncSetAttribute(sel_kernel_bf16<S, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
     if (e != cudaSuccess) return e;
-    const long long w = static_cast<long long>(a.H) * a.R;
+    const long long w = static_cast<long long>(a.H) * a.R * ((S * S + 15) / 16);
     EpiArgs none;
     memset(&none, 0, sizeof(none));
     sel_kernel_bf16<S, false><<<static_cast<unsigned>((w + SEL_WARPS - 1) / SEL_WARPS), SEL_WARPS * 32, sm, st>>>(a, none);
@@ -394,7 +410,7 @@ cudaError_t launch_sel_fused_s(const SelArgs& a, const EpiArgs& ep, cudaStream_t
   const int sm = SEL_WARPS * SEL_WARP_SMEM;
   cudaError_t e = cudaFuncSetAttribute(sel_kernel_bf16<S, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
   if (e != cudaSuccess) return e;
-  const long long w = static_cast<long long>(a.H) * a.R;
+  const long long w = static_cast<long long>(a.H) * a.R * ((S * S + 15) / 16);
   sel_kernel_bf16<S, true><<<static_cast<unsigned>((w + SEL_WARPS - 1) / SEL_WARPS), SEL_WARPS * 32, sm, st>>>(a, ep);
   return cudaGetLastError();
 }
@@ -406,6 +422,7 @@ cudaError_t launch_sel_fused(const SelArgs& a, const EpiArgs& ep, cudaStream_t s
     case 1: return launch_sel_fused_s<1>(a, ep, st);
     case 2: return launch_sel_fused_s<2>(a, ep, st);
     case 4: return launch_sel_fused_s<4>(a, ep, st);
+    case 8: return launch_sel_fused_s<8>(a, ep, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -415,9 +432,7 @@ cudaError_t launch_sel(const SelArgs& a, bool fp32, cudaStream_t st) {
     case 1: return launch_sel_s<1>(a, fp32, st);
     case 2: return launch_sel_s<2>(a, fp32, st);
     case 4: return launch_sel_s<4>(a, fp32, st);
-    case 8:
-      if (fp32) return launch_sel_s<8>(a, true, st);
-      return cudaErrorInvalidValue;
+    case 8: return launch_sel_s<8>(a, fp32, st);
     default: return cudaErrorInvalidValue;
   }
 }

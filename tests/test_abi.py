@@ -42,7 +42,6 @@ def _cfg(**kw):
     (dict(pad_h=10, grid_h=7), 2),                # a region row with no valid token
     (dict(pad_h=6, grid_h=8), 2),                 # pad smaller than the grid
     (dict(num_frames=0), 1),
-    (dict(dtype="bf16", pool_s=8, grid_h=16, grid_w=16), 3),
     (dict(fixed_frames=(0, 0)), 1),               # duplicated fixed frame
     (dict(fixed_frames=(5,)), 1),                 # fixed frame out of range
     (dict(fixed_frames=(0, 1, 2, 3)), 2),         # no candidate region left

@@ -17,9 +17,11 @@ S2_BF16 = GSAConfig("s2_bf16", 2, 10, 14, 10, 14, 1, 2, 64, 2, 12, "bf16")      
 PAD_VGGT_BF16 = GSAConfig("pad_vggt_bf16", 5, 10, 11, 12, 12, 3, 2, 64, 4, 6, "bf16", (0, 3))
 NO_SPECIAL_BF16 = GSAConfig("no_special_bf16", 4, 16, 16, 16, 16, 0, 1, 64, 4, 5, "bf16")
 PAD_F32 = GSAConfig("pad_vggt_f32", 4, 7, 7, 8, 8, 2, 2, 64, 2, 5, "fp32", (1,))
+S8_BF16 = GSAConfig("s8_bf16", 3, 16, 16, 16, 16, 2, 2, 64, 8, 3, "bf16")                  # 8x8 windows, R=12
+S8_PAD_BF16 = GSAConfig("s8_pad_bf16", 2, 14, 13, 16, 16, 1, 2, 64, 8, 2, "bf16")          # ragged 8x8 windows
 
 SMALL = [CONFIGS["tiny_fp32"], RAGGED_BF16, MULTI_TILE_BF16, S2_BF16, PAD_VGGT_BF16,
-         NO_SPECIAL_BF16, PAD_F32]
+         NO_SPECIAL_BF16, PAD_F32, S8_BF16, S8_PAD_BF16]
 
 
 def _cuda_inputs(cfg, seed=0):
