@@ -441,7 +441,8 @@ def run_b200(args, cfg, rank, world, local, dist):
     if args.ablations:
         ablations = {}
         specs = [("no_comp_value", dict(variant="no_comp_value")), ("no_selection", dict(variant="no_selection")),
-                 ("top8", dict(topk=8)), ("top16", dict(topk=16)), ("top64", dict(topk=64)), ("windows8x8", None)]
+                 ("top8", dict(topk=8)), ("top16", dict(topk=16)), ("top64", dict(topk=64)),
+                 ("flashvggt_descriptor_attention", dict(variant="descriptor")), ("windows8x8", None)]
         for name, kw in specs:
             if kw is None:
                 # 8x8 windows: the grid padded to a multiple of 8, inputs drawn for that layout
@@ -471,6 +472,12 @@ def run_b200(args, cfg, rank, world, local, dist):
                 raise RuntimeError(f"device status {st} in ablation {name}: {gsa.gsa_strerror(st)}")
             ams = max_over_ranks(a0.elapsed_time(a1) / 3, dist, dev)
             ablations[name] = {"ms": round(ams, 3), "vs_full": round(ams / ms, 3)}
+            if name == "flashvggt_descriptor_attention":
+                # every image and special token against (F * Hd * Wd descriptors + special tokens)
+                nd = cfg.num_frames * (cfg.grid_h // cfg.pool_s) * (cfg.grid_w // cfg.pool_s) + cfg.num_spec
+                fl = 4.0 * cfg.head_dim * cfg.num_heads * (cfg.num_frames * cfg.pad_h * cfg.pad_w + cfg.num_spec) * nd
+                tf = fl / (ams / 1e3) / 1e12
+                ablations[name].update({"tflops": round(tf, 1), "frac_of_sustained_bf16": round(tf / tpeak, 4)})
 
     if rank != 0:
         return None

@@ -76,10 +76,19 @@ extern "C" {
  *   GSA_VARIANT_NO_SELECTION   "移除选择分支": no top-k and no selection branch,
  *                              O_img = Upsample(O'_comp); sel_idx_out must be NULL
  * gate_mode is ignored by the two ablation variants; special tokens are
- * computed as in the full layer. */
+ * computed as in the full layer.
+ *   GSA_VARIANT_DESCRIPTOR     FlashVGGT's descriptor attention (a second method of
+ *                              the same pages, "FlashVGGT ... 描述符注意力"): every frame's
+ *                              valid K/V grid is resized bilinearly to
+ *                              (grid_h / pool_s, grid_w / pool_s) descriptors, and
+ *                              every image and special token attends to the
+ *                              descriptors of all frames plus all special tokens.
+ *                              topk, gate_mode and w_g are not used; sel_idx_out
+ *                              must be NULL. */
 #define GSA_VARIANT_FULL          0
 #define GSA_VARIANT_NO_COMP_VALUE 1
 #define GSA_VARIANT_NO_SELECTION  2
+#define GSA_VARIANT_DESCRIPTOR    3
 
 typedef struct gsa_ctx gsa_ctx;
 

@@ -19,7 +19,7 @@ GSA_OK = 0
 GSA_BF16, GSA_FP32 = 0, 1
 GSA_GATE_LEARNED, GSA_GATE_COMP_ONLY, GSA_GATE_SEL_ONLY = 0, 1, 2
 GATE_MODES = {"learned": 0, "comp_only": 1, "sel_only": 2}
-VARIANTS = {"full": 0, "no_comp_value": 1, "no_selection": 2}
+VARIANTS = {"full": 0, "no_comp_value": 1, "no_selection": 2, "descriptor": 3}
 GSA_PROFILE_TIMES, GSA_PROFILE_KEEP_OSEL = 1, 2
 EXPORTED = ("gsa_create", "gsa_workspace_bytes", "gsa_forward", "gsa_dense_forward",
             "gsa_get_intermediate", "gsa_set_profiling", "gsa_get_kernel_times",

@@ -35,7 +35,8 @@ int validate(const gsa_config* c, Derived* d) {
   if (c->num_fixed_frames < 0 || (c->num_fixed_frames > 0 && !c->fixed_frames))
     return GSA_ERR_INVALID_ARG;
   if (c->num_fixed_frames > GSA_MAX_FIXED_FRAMES) return GSA_ERR_UNSUPPORTED;
-  if (c->variant < GSA_VARIANT_FULL || c->variant > GSA_VARIANT_NO_SELECTION) return GSA_ERR_INVALID_ARG;
+  if (c->variant < GSA_VARIANT_FULL || c->variant > GSA_VARIANT_DESCRIPTOR) return GSA_ERR_INVALID_ARG;
+  if (c->variant == GSA_VARIANT_DESCRIPTOR && (c->grid_h < c->pool_s || c->grid_w < c->pool_s)) return GSA_ERR_SHAPE;
   if (!(c->softmax_scale >= 0.f) || isinf(c->softmax_scale)) return GSA_ERR_INVALID_ARG;
   if (c->head_dim != 64) return GSA_ERR_SHAPE;
   const int s = c->pool_s;
@@ -133,6 +134,14 @@ struct DeviceGuard {
     if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
   }
 };
+
+// the variants fix the blend: no compressed value -> O_sel, no selection ->
+// O_comp; the descriptor attention has no gate at all
+int effective_gate(const gsa_config& c) {
+  if (c.variant == GSA_VARIANT_NO_COMP_VALUE) return GSA_GATE_SEL_ONLY;
+  if (c.variant == GSA_VARIANT_NO_SELECTION || c.variant == GSA_VARIANT_DESCRIPTOR) return GSA_GATE_COMP_ONLY;
+  return c.gate_mode;
+}
 
 float scale_of(const gsa_config& c) {
   return c.softmax_scale > 0.f ? c.softmax_scale : 1.f / sqrtf(static_cast<float>(c.head_dim));
@@ -253,10 +262,8 @@ int forward_heads(gsa_ctx* c, int h0, int nh, const void* q_spec, const void* k_
   const gsa_config& cf = c->cfg;
   const Derived& d = c->d;
   // the ablation variants fix the blend: no compressed value -> O_sel, no selection -> O_comp
-  const int gate = cf.variant == GSA_VARIANT_NO_COMP_VALUE ? GSA_GATE_SEL_ONLY
-                   : cf.variant == GSA_VARIANT_NO_SELECTION ? GSA_GATE_COMP_ONLY
-                                                            : cf.gate_mode;
-  const bool no_sel = cf.variant == GSA_VARIANT_NO_SELECTION;
+  const int gate = effective_gate(cf);
+  const bool no_sel = cf.variant == GSA_VARIANT_NO_SELECTION || cf.variant == GSA_VARIANT_DESCRIPTOR;
   if (gate == GSA_GATE_LEARNED && !w_g) return GSA_ERR_INVALID_ARG;
   if (no_sel && sel_idx_out) return GSA_ERR_INVALID_ARG;
   const int H = nh;
@@ -297,6 +304,87 @@ int forward_heads(gsa_ctx* c, int h0, int nh, const void* q_spec, const void* k_
   if (!v_spec) v_spec = v_img;
   if (!w_g) w_g = q_img;         // never read when the gate is forced
   Prof prof(c, st, timing);
+
+  if (cf.variant == GSA_VARIANT_DESCRIPTOR) {
+    // FlashVGGT descriptor attention: descriptors of K and V into the pooled
+    // K/V workspace rows, then image queries and special queries attend to
+    // [descriptors of every frame ; special tokens of every frame]
+    const int Hd = cf.grid_h / cf.pool_s, Wd = cf.grid_w / cf.pool_s;
+    const long long ndesc = static_cast<long long>(cf.num_frames) * Hd * Wd;
+    // descriptors packed per head ([H][ndesc][64], ndesc <= R): the tensor-core
+    // attention addresses key rows as h * n_k + key
+    const long long rhs = ndesc * D;
+    DescArgs da;
+    da.src[0] = k_img; da.src[1] = v_img;
+    da.dst[0] = d.fp32 ? static_cast<void*>(comp32[1]) : static_cast<void*>(comp16[1]);
+    da.dst[1] = d.fp32 ? static_cast<void*>(comp32[2]) : static_cast<void*>(comp16[2]);
+    da.dst_hs = rhs;
+    da.H = H; da.F = cf.num_frames; da.Hp = cf.pad_h; da.Wp = cf.pad_w; da.Hv = cf.grid_h; da.Wv = cf.grid_w;
+    da.Hd = Hd; da.Wd = Wd;
+    if (launch_descriptors(da, d.fp32, st) != cudaSuccess) return GSA_ERR_CUDA;
+    prof.mark("descriptors");
+    const long long shs = d.spec_per_head * D, ihs = d.img_per_head * D;
+    const int spec_tiles = attn_tc_tiles(d.spec_per_head);
+    const int dtiles = attn_tc_tiles(ndesc);
+    for (int pass = 0; pass < 2; ++pass) {
+      // pass 0: image queries (one key split: plenty of CTAs); pass 1: special queries
+      if (pass == 1 && cf.num_special == 0) break;
+      const long long nq = pass == 0 ? d.img_per_head : d.spec_per_head;
+      const long long qhs = pass == 0 ? ihs : shs;
+      const void* qp = pass == 0 ? q_img : q_spec;
+      void* op = pass == 0 ? o_img : o_spec;
+      const int qmask = (pass == 0 && d.pads) ? MASK_IMG : MASK_NONE;
+      const int nseg = cf.num_special > 0 ? 2 : 1;
+      const int ttot = dtiles + (nseg > 1 ? spec_tiles : 0);
+      int tps = ttot, nsplit = 1;
+      if (pass == 1) {
+        attn_tc_split(H, nq, ttot, &tps, &nsplit);
+        const int cap = static_cast<int>((static_cast<long long>(d.spec_split) * cf.num_heads) / H);
+        if (nsplit > cap) {
+          tps = (ttot + cap - 1) / cap;
+          nsplit = (ttot + tps - 1) / tps;
+        }
+      }
+      if (!d.fp32) {
+        AttnArgs a;
+        memset(&a, 0, sizeof(a));
+        a.q = reinterpret_cast<const __nv_bfloat16*>(qp); a.q_hs = qhs; a.n_q = static_cast<int>(nq);
+        a.q_mask = qmask;
+        a.nseg = nseg;
+        a.k[0] = comp16[1]; a.v[0] = comp16[2]; a.kv_hs[0] = rhs; a.n_k[0] = static_cast<int>(ndesc);
+        a.kmask[0] = MASK_NONE;
+        a.k[1] = reinterpret_cast<const __nv_bfloat16*>(k_spec);
+        a.v[1] = reinterpret_cast<const __nv_bfloat16*>(v_spec);
+        a.kv_hs[1] = shs; a.n_k[1] = static_cast<int>(d.spec_per_head); a.kmask[1] = MASK_NONE;
+        a.tiles0 = dtiles; a.tiles_total = ttot; a.tiles_per_split = tps; a.n_split = nsplit;
+        a.H = H; a.g = g; a.scale_log2 = scale * LOG2E;
+        a.o16 = reinterpret_cast<__nv_bfloat16*>(op); a.o_hs = qhs;
+        a.part_o = c->at<float>(c->L.part_o); a.part_ml = c->at<float>(c->L.part_ml);
+        a.err = err;
+        if (launch_attn_tc(a, st) != cudaSuccess) return GSA_ERR_CUDA;
+        if (nsplit > 1) {
+          MergeArgs m;
+          m.part_o = a.part_o; m.part_ml = a.part_ml; m.n_split = nsplit; m.H = H;
+          m.n_q = a.n_q; m.scale_log2 = a.scale_log2; m.o16 = a.o16; m.o32 = nullptr; m.o_hs = qhs;
+          if (launch_merge(m, st) != cudaSuccess) return GSA_ERR_CUDA;
+        }
+      } else {
+        AttnF32Args a;
+        memset(&a, 0, sizeof(a));
+        a.q = reinterpret_cast<const float*>(qp); a.q_hs = qhs; a.n_q = static_cast<int>(nq); a.q_mask = qmask;
+        a.nseg = nseg;
+        a.k[0] = comp32[1]; a.v[0] = comp32[2]; a.kv_hs[0] = rhs; a.n_k[0] = static_cast<int>(ndesc);
+        a.kmask[0] = MASK_NONE;
+        a.k[1] = reinterpret_cast<const float*>(k_spec); a.v[1] = reinterpret_cast<const float*>(v_spec);
+        a.kv_hs[1] = shs; a.n_k[1] = static_cast<int>(d.spec_per_head); a.kmask[1] = MASK_NONE;
+        a.H = H; a.g = g; a.scale = scale;
+        a.o = reinterpret_cast<float*>(op); a.o_hs = qhs;
+        if (launch_attn_f32(a, false, st) != cudaSuccess) return GSA_ERR_CUDA;
+      }
+      prof.mark(pass == 0 ? "descriptor_attn_img" : "descriptor_attn_spec");
+    }
+    return GSA_OK;
+  }
 
   // K1 pool
   PoolArgs pa;
@@ -450,9 +538,7 @@ int gsa_forward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void* 
   if (!c || !q_img || !k_img || !v_img || !o_img) return GSA_ERR_INVALID_ARG;
   const gsa_config& cf = c->cfg;
   if (cf.num_special > 0 && (!q_spec || !k_spec || !v_spec || !o_spec)) return GSA_ERR_INVALID_ARG;
-  const int gate = cf.variant == GSA_VARIANT_NO_COMP_VALUE ? GSA_GATE_SEL_ONLY
-                   : cf.variant == GSA_VARIANT_NO_SELECTION ? GSA_GATE_COMP_ONLY
-                                                            : cf.gate_mode;
+  const int gate = effective_gate(cf);
   if (gate == GSA_GATE_LEARNED && !w_g) return GSA_ERR_INVALID_ARG;
   if (cf.variant == GSA_VARIANT_NO_SELECTION && sel_idx_out) return GSA_ERR_INVALID_ARG;
   DeviceGuard dg(c->device);
@@ -470,9 +556,7 @@ int gsa_forward_host(gsa_ctx* c, const void* q_spec, const void* k_spec, const v
   const Derived& d = c->d;
   const bool spec = cf.num_special > 0;
   if (spec && (!q_spec || !k_spec || !v_spec || !o_spec)) return GSA_ERR_INVALID_ARG;
-  const int gate = cf.variant == GSA_VARIANT_NO_COMP_VALUE ? GSA_GATE_SEL_ONLY
-                   : cf.variant == GSA_VARIANT_NO_SELECTION ? GSA_GATE_COMP_ONLY
-                                                            : cf.gate_mode;
+  const int gate = effective_gate(cf);
   if (gate == GSA_GATE_LEARNED && !w_g) return GSA_ERR_INVALID_ARG;
   if (cf.variant == GSA_VARIANT_NO_SELECTION && sel_idx_out) return GSA_ERR_INVALID_ARG;
   DeviceGuard dg(c->device);

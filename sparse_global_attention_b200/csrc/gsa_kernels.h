@@ -17,6 +17,15 @@ struct PoolArgs {
 };
 cudaError_t launch_pool(const PoolArgs& a, bool fp32, cudaStream_t st);
 
+// ---- FlashVGGT descriptors: bilinear resize of K/V to (Hv/r, Wv/r) per frame --
+struct DescArgs {
+  const void* src[2];        // K, V image tokens [H][F][Hp][Wp][64]
+  void* dst[2];              // descriptors [H][F][Hd][Wd][64] (head stride dst_hs), context dtype
+  long long dst_hs;          // elements per head in dst
+  int H, F, Hp, Wp, Hv, Wv, Hd, Wd;
+};
+cudaError_t launch_descriptors(const DescArgs& a, bool fp32, cudaStream_t st);
+
 // ---- attention core (K2 compressed + top-k, K5 special, K6 dense) ----------
 struct AttnArgs {
   const __nv_bfloat16* q;    // [H][n_q][64]

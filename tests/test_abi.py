@@ -47,7 +47,7 @@ def _cfg(**kw):
     (dict(fixed_frames=(0, 1, 2, 3)), 2),         # no candidate region left
     (dict(gate_mode=7), 1),
     (dict(softmax_scale=-1.0), 1),
-    (dict(variant=3), 1),                         # no such ablation variant
+    (dict(variant=4), 1),                         # no such variant
     (dict(variant=-1), 1),
 ])
 def test_invalid_configs_are_rejected_on_the_host(kw, code):
