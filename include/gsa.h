@@ -140,6 +140,28 @@ GSA_API int gsa_forward(gsa_ctx *ctx,
                 const void *w_g, void *o_spec, void *o_img, int32_t *sel_idx_out,
                 void *stream);
 
+/* Backward pass of gsa_forward ("Speed3R ... GSA": the notes train the layer
+ * end to end; the region selection is a discrete choice and gets no gradient).
+ * Call on the same context after gsa_forward with the same inputs: the
+ * forward's pooled tensors, O'_comp, selection and softmax statistics are read
+ * from the workspace.  o_spec is the forward's special-token output;
+ * d_o_spec / d_o_img are the output gradients (context dtype, layouts of
+ * o_spec / o_img).  Writes float32 gradients, the layouts of the inputs:
+ * dq/dk/dv_img [H][F][pad_h][pad_w][64] (0 on pads), dq/dk/dv_spec
+ * [H][F][num_special][64] (unused when num_special = 0), dw_g [H][64][64]
+ * (0 when the gate is forced).  bf16 contexts of the full layer with
+ * pool_s <= 4 only (GSA_ERR_UNSUPPORTED otherwise); allocates a scratch of
+ * about 5 x H x R x 256 bytes plus one float per image-token channel on first
+ * use (GSA_ERR_OOM if that fails), freed by gsa_destroy.  Asynchronous on
+ * `stream`. */
+GSA_API int gsa_backward(gsa_ctx *ctx,
+                         const void *q_spec, const void *k_spec, const void *v_spec,
+                         const void *q_img, const void *k_img, const void *v_img,
+                         const void *w_g, const void *o_spec,
+                         const void *d_o_spec, const void *d_o_img,
+                         float *dq_spec, float *dk_spec, float *dv_spec,
+                         float *dq_img, float *dk_img, float *dv_img, float *dw_g, void *stream);
+
 /* gsa_forward with HOST buffers: the same arguments and layouts, every tensor
  * pointer (inputs, outputs, optional sel_idx_out) in host memory.  The heads
  * are processed in up to eight chunks: the host-to-device copies of chunk i+1

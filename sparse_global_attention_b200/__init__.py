@@ -24,7 +24,7 @@ GSA_PROFILE_TIMES, GSA_PROFILE_KEEP_OSEL = 1, 2
 EXPORTED = ("gsa_create", "gsa_workspace_bytes", "gsa_forward", "gsa_dense_forward",
             "gsa_get_intermediate", "gsa_set_profiling", "gsa_get_kernel_times",
             "gsa_get_status", "gsa_strerror", "gsa_destroy", "gsa_special_attention_noalloc",
-            "gsa_debug_expire_wait", "gsa_forward_host")
+            "gsa_debug_expire_wait", "gsa_forward_host", "gsa_backward")
 
 
 class gsa_config(ctypes.Structure):
@@ -264,6 +264,27 @@ class GSALayer:
                   hout["o_img"].data_ptr(), None if sel_idx is None else sel_idx.data_ptr(), st or None),
                "gsa_forward_host")
         return hout
+
+    def backward(self, x, out, dout, stream=None):
+        """gsa_backward after forward(x) -> out: dout = {"o_img", "o_spec"} output
+        gradients (context dtype).  Returns float32 gradients of every input:
+        dq_img, dk_img, dv_img, dq_spec, dk_spec, dv_spec, dw_g."""
+        import torch
+        st = stream if stream is not None else torch.cuda.current_stream().cuda_stream
+        gr = {"dq_img": x["q_img"], "dk_img": x["k_img"], "dv_img": x["v_img"], "dq_spec": x["q_spec"],
+              "dk_spec": x["k_spec"], "dv_spec": x["v_spec"], "dw_g": x["w_g"]}
+        gr = {k: torch.empty(v.shape, dtype=torch.float32, device=v.device) for k, v in gr.items()}
+        has_spec = x["q_spec"].numel() > 0
+        p = lambda t: t.data_ptr() if (t is not None and t.numel() > 0) else None
+        fn = load_library().gsa_backward
+        fn.argtypes = [ctypes.c_void_p] * 19
+        fn.restype = ctypes.c_int
+        _check(fn(self.ctx, p(x["q_spec"]), p(x["k_spec"]), p(x["v_spec"]), p(x["q_img"]), p(x["k_img"]),
+                  p(x["v_img"]), p(x["w_g"]), p(out["o_spec"]) if has_spec else None,
+                  p(dout["o_spec"]) if has_spec else None, p(dout["o_img"]),
+                  p(gr["dq_spec"]), p(gr["dk_spec"]), p(gr["dv_spec"]), p(gr["dq_img"]), p(gr["dk_img"]),
+                  p(gr["dv_img"]), p(gr["dw_g"]), st or None), "gsa_backward")
+        return gr
 
     def dense(self, q, k, v, o=None, stream=None):
         import torch

@@ -607,6 +607,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (GO) {
         // guide only: no attention output
       } else if (a.n_split == 1) {
+        if (a.lse) a.lse[static_cast<long long>(h) * a.n_q + row] = l > 0.f ? m * sl2 + __log2f(l) : -INFINITY;
         float inv = l > 0.f ? 1.f / l : 0.f;
         if (a.q_mask != MASK_NONE && !key_valid(a.q_mask, a.g, row)) inv = 0.f;
         const long long base = h * a.o_hs + static_cast<long long>(row) * D;

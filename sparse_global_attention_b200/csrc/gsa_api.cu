@@ -75,7 +75,7 @@ int validate(const gsa_config* c, Derived* d) {
 }
 
 struct Layout {
-  size_t comp16[3], complo[2], comp32[3], ocomp, idx, osel, part_o, part_ml, err, total;
+  size_t comp16[3], complo[2], comp32[3], ocomp, idx, osel, part_o, part_ml, lse_c, lse_s, err, total;
 };
 
 Layout make_layout(const gsa_config* c, const Derived& d) {
@@ -92,6 +92,8 @@ Layout make_layout(const gsa_config* c, const Derived& d) {
   const size_t sp = static_cast<size_t>(d.spec_split > 1 ? d.spec_split : 0) * c->num_heads * d.spec_per_head;
   L.part_o = take(sp * D * 4);
   L.part_ml = take(sp * 2 * 4);
+  L.lse_c = take(rows * 4);                                                  // for the backward
+  L.lse_s = take(static_cast<size_t>(c->num_heads) * d.spec_per_head * 4);
   L.err = take(16);
   L.total = off;
   return L;
@@ -115,6 +117,8 @@ struct gsa_ctx {
   // outputs, copy streams and per-chunk events, created on first use
   uint8_t* stage;
   size_t stage_bytes;
+  uint8_t* bw;                 // backward scratch (gsa_backward), created on first use
+  size_t bw_bytes;
   cudaStream_t s_in, s_out;
   cudaEvent_t ev_start, ev_in[MAX_CHUNKS], ev_comp[MAX_CHUNKS], ev_out;
   template <typename T>
@@ -232,6 +236,7 @@ int gsa_create(const gsa_config* cfg, gsa_ctx** out) {
 void gsa_destroy(gsa_ctx* c) {
   if (!c) return;
   DeviceGuard dg(c->device);
+  if (c->bw) cudaFree(c->bw);
   if (c->stage) {
     cudaFree(c->stage);
     cudaStreamDestroy(c->s_in);
@@ -364,6 +369,7 @@ int forward_heads(gsa_ctx* c, int h0, int nh, const void* q_spec, const void* k_
         if (launch_attn_tc(a, st) != cudaSuccess) return GSA_ERR_CUDA;
         if (nsplit > 1) {
           MergeArgs m;
+          m.lse = nullptr;
           m.part_o = a.part_o; m.part_ml = a.part_ml; m.n_split = nsplit; m.H = H;
           m.n_q = a.n_q; m.scale_log2 = a.scale_log2; m.o16 = a.o16; m.o32 = nullptr; m.o_hs = qhs;
           if (launch_merge(m, st) != cudaSuccess) return GSA_ERR_CUDA;
@@ -416,6 +422,7 @@ int forward_heads(gsa_ctx* c, int h0, int nh, const void* q_spec, const void* k_
     a.o32 = ocomp; a.o_hs = rhs;
     a.kc = no_sel ? 0 : d.kc; a.cand = idx; a.cand_user = sel_idx_out;
     a.guide_only = cf.variant == GSA_VARIANT_NO_COMP_VALUE ? 1 : 0;
+    a.lse = reinterpret_cast<float*>(ws(c->L.lse_c, static_cast<size_t>(d.R) * 4));
     a.rpf = d.rpf; a.n_fixed = cf.num_fixed_frames;
     for (int i = 0; i < cf.num_fixed_frames; ++i) a.fixed[i] = c->fixed[i];
     a.err = err;
@@ -498,13 +505,16 @@ int forward_heads(gsa_ctx* c, int h0, int nh, const void* q_spec, const void* k_
       a.H = H; a.g = g; a.scale_log2 = scale * LOG2E;
       a.o16 = reinterpret_cast<__nv_bfloat16*>(o_spec); a.o_hs = shs;
       a.part_o = c->at<float>(c->L.part_o); a.part_ml = c->at<float>(c->L.part_ml);
+      a.lse = reinterpret_cast<float*>(ws(c->L.lse_s, static_cast<size_t>(d.spec_per_head) * 4));
       a.err = err;
       if (launch_attn_tc(a, st) != cudaSuccess) return GSA_ERR_CUDA;
       prof.mark("special");
       if (nsplit > 1) {
         MergeArgs m;
+        m.lse = nullptr;
         m.part_o = a.part_o; m.part_ml = a.part_ml; m.n_split = nsplit; m.H = H;
         m.n_q = a.n_q; m.scale_log2 = a.scale_log2; m.o16 = a.o16; m.o32 = nullptr; m.o_hs = shs;
+        m.lse = a.lse;
         if (launch_merge(m, st) != cudaSuccess) return GSA_ERR_CUDA;
         prof.mark("special_merge");
       }
@@ -630,6 +640,139 @@ int gsa_forward_host(gsa_ctx* c, const void* q_spec, const void* k_spec, const v
   if (cudaEventRecord(c->ev_out, c->s_out) != cudaSuccess) return GSA_ERR_CUDA;
   if (cudaStreamWaitEvent(st, c->ev_out, 0) != cudaSuccess) return GSA_ERR_CUDA;
   c->last_stream = st;
+  return GSA_OK;
+}
+
+int gsa_backward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void* v_spec, const void* q_img,
+                 const void* k_img, const void* v_img, const void* w_g, const void* o_spec, const void* d_o_spec,
+                 const void* d_o_img, float* dq_spec, float* dk_spec, float* dv_spec, float* dq_img, float* dk_img,
+                 float* dv_img, float* dw_g, void* stream) {
+  if (!c || !q_img || !k_img || !v_img || !d_o_img || !dq_img || !dk_img || !dv_img || !dw_g)
+    return GSA_ERR_INVALID_ARG;
+  const gsa_config& cf = c->cfg;
+  const Derived& d = c->d;
+  const bool spec = cf.num_special > 0;
+  if (spec && (!q_spec || !k_spec || !v_spec || !o_spec || !d_o_spec || !dq_spec || !dk_spec || !dv_spec))
+    return GSA_ERR_INVALID_ARG;
+  if (d.fp32 || cf.variant != GSA_VARIANT_FULL || cf.pool_s > 4) return GSA_ERR_UNSUPPORTED;
+  const int gate = effective_gate(cf);
+  if (gate == GSA_GATE_LEARNED && !w_g) return GSA_ERR_INVALID_ARG;
+  if (cf.num_fixed_frames > 0 && !spec) return GSA_ERR_INVALID_ARG;
+  DeviceGuard dg(c->device);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  c->last_stream = st;
+  const int H = cf.num_heads;
+  const size_t rows = static_cast<size_t>(H) * d.R;
+  const size_t img = static_cast<size_t>(H) * d.img_per_head;
+  const size_t sp = static_cast<size_t>(H) * d.spec_per_head;
+  // scratch: dO'_comp fp32 + bf16, D of compressed and special rows, dQ/dK/dV_comp, da
+  size_t off[8], tot = 0;
+  const size_t sz[8] = {rows * D * 4, rows * D * 2, rows * 4, sp * 4, rows * D * 4, rows * D * 4, rows * D * 4,
+                        img * D * 4};
+  for (int i = 0; i < 8; ++i) {
+    off[i] = tot;
+    tot = align_up(tot + sz[i]);
+  }
+  if (!c->bw) {
+    if (cudaMalloc(&c->bw, tot) != cudaSuccess) {
+      c->bw = nullptr;
+      return GSA_ERR_OOM;
+    }
+    c->bw_bytes = tot;
+  }
+  float* docomp = reinterpret_cast<float*>(c->bw + off[0]);
+  __nv_bfloat16* docomp16 = reinterpret_cast<__nv_bfloat16*>(c->bw + off[1]);
+  float* Dc = reinterpret_cast<float*>(c->bw + off[2]);
+  float* Ds = reinterpret_cast<float*>(c->bw + off[3]);
+  float* dqc = reinterpret_cast<float*>(c->bw + off[4]);
+  float* dkc = reinterpret_cast<float*>(c->bw + off[5]);
+  float* dvc = reinterpret_cast<float*>(c->bw + off[6]);
+  float* da = reinterpret_cast<float*>(c->bw + off[7]);
+  const Grid g = grid_of(cf);
+  const float scale = scale_of(cf);
+  int* err = c->at<int>(c->L.err);
+  if (!k_spec) k_spec = k_img;
+  if (!v_spec) v_spec = v_img;
+  if (!w_g) w_g = q_img;
+  // gradients reached by atomics or accumulation start at zero
+  if (cudaMemsetAsync(dk_img, 0, img * D * 4, st) != cudaSuccess || cudaMemsetAsync(dv_img, 0, img * D * 4, st) != cudaSuccess)
+    return GSA_ERR_CUDA;
+  if (spec && (cudaMemsetAsync(dk_spec, 0, sp * D * 4, st) != cudaSuccess ||
+               cudaMemsetAsync(dv_spec, 0, sp * D * 4, st) != cudaSuccess))
+    return GSA_ERR_CUDA;
+
+  // 1. selection branch and gate (windows), dO'_comp, dq of the image tokens
+  SelBwdArgs sb;
+  memset(&sb, 0, sizeof(sb));
+  SelArgs& sa = sb.s;
+  sa.q_img = q_img; sa.k_img = k_img; sa.v_img = v_img; sa.k_spec = k_spec; sa.v_spec = v_spec;
+  sa.idx = c->at<int>(c->L.idx); sa.o_sel = nullptr;
+  sa.H = H; sa.F = cf.num_frames; sa.R = d.R; sa.rpf = d.rpf; sa.topk = cf.topk; sa.s = cf.pool_s;
+  sa.g = g; sa.scale_log2 = scale * LOG2E; sa.n_fixed = cf.num_fixed_frames;
+  for (int i = 0; i < cf.num_fixed_frames; ++i) sa.fixed[i] = c->fixed[i];
+  sa.err = err;
+  sb.w_g = w_g; sb.o_comp = c->at<float>(c->L.ocomp); sb.d_o = reinterpret_cast<const __nv_bfloat16*>(d_o_img);
+  sb.gate_mode = gate; sb.dq = dq_img; sb.dk = dk_img; sb.dv = dv_img;
+  sb.dk_spec = spec ? dk_spec : nullptr; sb.dv_spec = spec ? dv_spec : nullptr;
+  sb.d_ocomp = docomp; sb.da = da;
+  if (launch_sel_bwd(sb, st) != cudaSuccess) return GSA_ERR_CUDA;
+
+  // 2. compressed attention (split guide scores, as in the forward)
+  const long long rhs = static_cast<long long>(d.R) * D;
+  if (launch_rowdot(docomp, nullptr, c->at<float>(c->L.ocomp), nullptr, static_cast<long long>(rows), Dc, docomp16,
+                    st) != cudaSuccess)
+    return GSA_ERR_CUDA;
+  BwdArgs ba;
+  memset(&ba, 0, sizeof(ba));
+  ba.q = c->at<__nv_bfloat16>(c->L.comp16[0]); ba.q_lo = c->at<__nv_bfloat16>(c->L.complo[0]);
+  ba.k_lo = c->at<__nv_bfloat16>(c->L.complo[1]); ba.q_hs = rhs; ba.n_q = d.R; ba.nseg = 1;
+  ba.k[0] = c->at<__nv_bfloat16>(c->L.comp16[1]); ba.v[0] = c->at<__nv_bfloat16>(c->L.comp16[2]);
+  ba.kv_hs[0] = rhs; ba.n_k[0] = d.R; ba.kmask[0] = MASK_NONE;
+  ba.dO = docomp16; ba.do_hs = rhs; ba.lse2 = c->at<float>(c->L.lse_c); ba.Dv = Dc;
+  ba.dq = dqc; ba.dq_hs = rhs; ba.dq_accum = 0;
+  ba.dk[0] = dkc; ba.dv[0] = dvc; ba.dkv_hs[0] = rhs; ba.dkv_accum = 0;
+  ba.H = H; ba.g = g; ba.scale_log2 = scale * LOG2E; ba.scale = scale;
+  if (launch_attn_bwd(ba, st) != cudaSuccess) return GSA_ERR_CUDA;
+
+  // 3. pooling: each valid token takes its region's gradient over the region's size
+  PoolBwdArgs pb;
+  pb.dcomp[0] = dqc; pb.dcomp[1] = dkc; pb.dcomp[2] = dvc;
+  pb.dimg[0] = dq_img; pb.dimg[1] = dk_img; pb.dimg[2] = dv_img;
+  pb.H = H; pb.F = cf.num_frames; pb.Hp = cf.pad_h; pb.Wp = cf.pad_w; pb.Hv = cf.grid_h; pb.Wv = cf.grid_w;
+  pb.s = cf.pool_s;
+  if (launch_pool_bwd(pb, st) != cudaSuccess) return GSA_ERR_CUDA;
+
+  // 4. special tokens over every special and valid image token
+  if (spec) {
+    const long long shs = d.spec_per_head * D, ihs = d.img_per_head * D;
+    if (launch_rowdot(nullptr, reinterpret_cast<const __nv_bfloat16*>(d_o_spec), nullptr,
+                      reinterpret_cast<const __nv_bfloat16*>(o_spec), static_cast<long long>(sp), Ds, nullptr,
+                      st) != cudaSuccess)
+      return GSA_ERR_CUDA;
+    BwdArgs bs;
+    memset(&bs, 0, sizeof(bs));
+    bs.q = reinterpret_cast<const __nv_bfloat16*>(q_spec); bs.q_hs = shs; bs.n_q = static_cast<int>(d.spec_per_head);
+    bs.nseg = 2;
+    bs.k[0] = reinterpret_cast<const __nv_bfloat16*>(k_spec); bs.v[0] = reinterpret_cast<const __nv_bfloat16*>(v_spec);
+    bs.kv_hs[0] = shs; bs.n_k[0] = static_cast<int>(d.spec_per_head); bs.kmask[0] = MASK_NONE;
+    bs.k[1] = reinterpret_cast<const __nv_bfloat16*>(k_img); bs.v[1] = reinterpret_cast<const __nv_bfloat16*>(v_img);
+    bs.kv_hs[1] = ihs; bs.n_k[1] = static_cast<int>(d.img_per_head); bs.kmask[1] = d.pads ? MASK_IMG : MASK_NONE;
+    bs.dO = reinterpret_cast<const __nv_bfloat16*>(d_o_spec); bs.do_hs = shs;
+    bs.lse2 = c->at<float>(c->L.lse_s); bs.Dv = Ds;
+    bs.dq = dq_spec; bs.dq_hs = shs; bs.dq_accum = 0;
+    bs.dk[0] = dk_spec; bs.dv[0] = dv_spec; bs.dkv_hs[0] = shs;
+    bs.dk[1] = dk_img; bs.dv[1] = dv_img; bs.dkv_hs[1] = ihs; bs.dkv_accum = 1;
+    bs.H = H; bs.g = g; bs.scale_log2 = scale * LOG2E; bs.scale = scale;
+    if (launch_attn_bwd(bs, st) != cudaSuccess) return GSA_ERR_CUDA;
+  }
+
+  // 5. the gate matrix
+  if (gate == GSA_GATE_LEARNED) {
+    if (launch_dwg(da, reinterpret_cast<const __nv_bfloat16*>(q_img), H, d.img_per_head, dw_g, st) != cudaSuccess)
+      return GSA_ERR_CUDA;
+  } else if (cudaMemsetAsync(dw_g, 0, static_cast<size_t>(H) * D * D * 4, st) != cudaSuccess) {
+    return GSA_ERR_CUDA;
+  }
   return GSA_OK;
 }
 

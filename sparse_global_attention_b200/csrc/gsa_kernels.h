@@ -41,6 +41,7 @@ struct AttnArgs {
   int n_k[2];
   int kmask[2];              // MaskMode per segment
   int guide_only;            // top-k only: S and the top-k, no P V and no output
+  float* lse;                // optional [H][n_q] base-2 log-sum-exp per row (n_split == 1)
   int tiles0;                // 128-key tiles of segment 0
   int tiles_total;
   int tiles_per_split;
@@ -62,7 +63,6 @@ struct AttnArgs {
   int fixed[MAX_FIXED];      // frames excluded from the candidates
   int* err;                  // device error word
 };
-cudaError_t launch_attn(const AttnArgs& a, bool topk, cudaStream_t st);
 // tcgen05/TMEM/TMA version: 2 x 128 query rows per CTA, 128-key tiles; the
 // top-k runs when a.kc > 0 (a.q_lo / a.k_lo required)
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st);
@@ -79,6 +79,7 @@ struct MergeArgs {
   __nv_bfloat16* o16;
   float* o32;
   long long o_hs;
+  float* lse;                // optional [H][n_q] base-2 log-sum-exp of each row (backward)
 };
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t st);
 
@@ -132,5 +133,68 @@ cudaError_t launch_attn_f32(const AttnF32Args& a, bool topk, cudaStream_t st);
 // one CTA waits on an mbarrier that nothing completes, gives up after limit_ns
 // of global time and records the timeout code in *err
 cudaError_t launch_expire_wait(int* err, unsigned long long limit_ns, cudaStream_t st);
+
+// ---- backward ----------------------------------------------------------------
+// dense attention backward (flash style) for one query set against up to two
+// key segments; P is recomputed from the forward's base-2 log-sum-exp
+struct BwdArgs {
+  const __nv_bfloat16* q;    // [H][n_q][64]
+  const __nv_bfloat16* q_lo; // optional low parts of q and k[0] (split scores), else nullptr
+  const __nv_bfloat16* k_lo;
+  long long q_hs;
+  int n_q;
+  int nseg;
+  const __nv_bfloat16* k[2];
+  const __nv_bfloat16* v[2];
+  long long kv_hs[2];
+  int n_k[2];
+  int kmask[2];
+  const __nv_bfloat16* dO;   // [H][n_q][64]
+  long long do_hs;
+  const float* lse2;         // [H][n_q] log2 sum exp2(S * scale_log2)
+  const float* Dv;           // [H][n_q] rowsum(dO o O)
+  float* dq;                 // [H][n_q][64] fp32
+  long long dq_hs;
+  int dq_accum;              // 1: add to dq, 0: overwrite
+  float* dk[2];              // [H][n_k][64] fp32 per segment (nullptr: skip the segment)
+  float* dv[2];
+  long long dkv_hs[2];
+  int dkv_accum;
+  int H;
+  Grid g;
+  float scale_log2, scale;
+};
+cudaError_t launch_attn_bwd(const BwdArgs& a, cudaStream_t st);
+
+// selection + gate backward: one warp per window (s <= 4)
+struct SelBwdArgs {
+  SelArgs s;                 // the forward's selection arguments (o_sel unused)
+  const void* w_g;
+  const float* o_comp;       // O'_comp [H][R][64]
+  const __nv_bfloat16* d_o;  // dO_img [H][F][Hp][Wp][64]
+  int gate_mode;
+  float* dq;                 // fp32 [H][F][Hp][Wp][64]: written (window tokens)
+  float* dk;                 // fp32 image-token dK/dV: atomically added
+  float* dv;
+  float* dk_spec;            // fp32 [H][F][ns][64] (fixed-frame special keys): atomically added
+  float* dv_spec;
+  float* d_ocomp;            // fp32 [H][R][64]: written
+  float* da;                 // fp32 [H][F][Hp][Wp][64]: gate pre-activation gradient (0 on pads)
+};
+cudaError_t launch_sel_bwd(const SelBwdArgs& a, cudaStream_t st);
+
+// pool backward and small steps
+struct PoolBwdArgs {
+  const float* dcomp[3];     // dQ_comp, dK_comp, dV_comp [H][R][64]
+  float* dimg[3];            // += into [H][F][Hp][Wp][64]
+  int H, F, Hp, Wp, Hv, Wv, s;
+};
+cudaError_t launch_pool_bwd(const PoolBwdArgs& a, cudaStream_t st);
+// D[h][i] = sum_c dO[h][i][c] * O[h][i][c]; dO fp32 or bf16 (do32 / do16), O fp32 or bf16;
+// optional bf16 copy of a fp32 dO
+cudaError_t launch_rowdot(const float* do32, const __nv_bfloat16* do16, const float* o32, const __nv_bfloat16* o16,
+                          long long rows, float* D, __nv_bfloat16* do16_out, cudaStream_t st);
+// dW_g[h] = sum over tokens of da (x) q  ([H][64][64], fp32, overwritten)
+cudaError_t launch_dwg(const float* da, const __nv_bfloat16* q, int H, long long tokens, float* dwg, cudaStream_t st);
 
 }  // namespace gsa

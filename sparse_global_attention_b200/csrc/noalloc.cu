@@ -103,6 +103,7 @@ extern "C" int gsa_special_attention_noalloc(const void* q_spec, const void* k_s
   if (launch_attn_tc(a, st) != cudaSuccess) return GSA_ERR_CUDA;
   if (n_split > 1) {
     MergeArgs m;
+    m.lse = nullptr;
     m.part_o = part_o; m.part_ml = part_ml; m.n_split = n_split; m.H = num_heads;
     m.n_q = static_cast<int>(M); m.scale_log2 = a.scale_log2; m.o16 = a.o16; m.o32 = nullptr; m.o_hs = M * D;
     if (launch_merge(m, st) != cudaSuccess) return GSA_ERR_CUDA;

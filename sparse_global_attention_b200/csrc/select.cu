@@ -438,3 +438,449 @@ cudaError_t launch_sel(const SelArgs& a, bool fp32, cudaStream_t st) {
 }
 
 }  // namespace gsa
+
+// ---- backward: selection branch and gate, one warp per window (s <= 4) ----------
+// Per-warp shared memory: Q (2 KB) | 2 stages x (K 4 KB | V 4 KB) | dO_sel tile
+// (2 KB, bf16, swizzled) | dS^T and P^T tiles ([32 keys][16 queries] bf16) |
+// region table | key validity.
+namespace gsa {
+namespace {
+
+constexpr int SB_Q = 0;
+constexpr int SB_KV = 16 * 128;
+constexpr int SB_DO = SB_KV + 4 * SEL_TILE;
+constexpr int SB_DST = SB_DO + 16 * 128;
+constexpr int SB_PT = SB_DST + SEL_BN * 32;
+constexpr int SB_REG = SB_PT + SEL_BN * 32;
+constexpr int SB_VAL = SB_REG + KC_MAX * 8;
+constexpr int SB_WARP = (SB_VAL + 2 * SEL_BN + 127) / 128 * 128;
+
+// A fragments (m16 x k16) of rows [r0, r0 + 16) of a [rows][16] bf16 tile with a 32-byte pitch
+__device__ __forceinline__ void ldsm_pitch32(uint32_t base, int r0, uint32_t (&a)[4]) {
+  const int lane = threadIdx.x & 31, j = lane >> 3;
+  const uint32_t addr = base + (r0 + (j & 1) * 8 + (lane & 7)) * 32 + (j >> 1) * 16;
+  ldsm_x4(addr, a[0], a[1], a[2], a[3]);
+}
+
+template <int S>
+__global__ void __launch_bounds__(SEL_WARPS * 32) sel_bwd_kernel(const SelBwdArgs b) {
+  const SelArgs& a = b.s;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3, mi = lane >> 3, lr = lane & 7;
+  uint8_t* wbase = smem + warp * SB_WARP;
+  const uint32_t sQ = smem_u32(wbase) + SB_Q;
+  const uint32_t sKV = smem_u32(wbase) + SB_KV;
+  const uint32_t sdO = smem_u32(wbase) + SB_DO;
+  __nv_bfloat16* sdSt = reinterpret_cast<__nv_bfloat16*>(wbase + SB_DST);
+  __nv_bfloat16* sPt = reinterpret_cast<__nv_bfloat16*>(wbase + SB_PT);
+  int2* sReg = reinterpret_cast<int2*>(wbase + SB_REG);
+  uint8_t* sValid = wbase + SB_VAL;
+
+  const long long win = static_cast<long long>(blockIdx.x) * SEL_WARPS + warp;
+  if (win >= static_cast<long long>(a.H) * a.R) return;      // warp-uniform
+  const int h = static_cast<int>(win / a.R);
+  const int r = static_cast<int>(win - static_cast<long long>(h) * a.R);
+  const long long img_hs = static_cast<long long>(a.F) * a.g.Hp * a.g.Wp * D;
+  const long long spec_hs = static_cast<long long>(a.F) * a.g.ns * D;
+  const __nv_bfloat16* qh = reinterpret_cast<const __nv_bfloat16*>(a.q_img) + h * img_hs;
+  const __nv_bfloat16* kh = reinterpret_cast<const __nv_bfloat16*>(a.k_img) + h * img_hs;
+  const __nv_bfloat16* vh = reinterpret_cast<const __nv_bfloat16*>(a.v_img) + h * img_hs;
+  const __nv_bfloat16* ksh = reinterpret_cast<const __nv_bfloat16*>(a.k_spec) + h * spec_hs;
+  const __nv_bfloat16* vsh = reinterpret_cast<const __nv_bfloat16*>(a.v_spec) + h * spec_hs;
+  const int f = r / a.rpf, rr0 = r - f * a.rpf;
+  const int rx = a.g.Wp / S;
+  const int wi = rr0 / rx, wj = rr0 - wi * rx;
+  for (int j = lane; j < a.topk; j += 32) {
+    int v = a.idx[win * a.topk + j];
+    if (v < 0 || v >= a.R) {
+      set_error(a.err, ERR_BOUNDS);
+      v = 0;
+    }
+    sReg[j] = region_base<S>(a, v);
+  }
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int e = lane + 32 * it;
+    const int row = e >> 3, c = e & 7;
+    const int y = wi * S + row / S, x = wj * S + row % S;
+    const bool ok = row < S * S && y < a.g.Hv && x < a.g.Wv;
+    const long long tok = ok ? (static_cast<long long>(f) * a.g.Hp + y) * a.g.Wp + x : 0;
+    cp_async16(sQ + swz(row, c), qh + tok * D + c * 8, ok ? 16 : 0);
+  }
+  cp_async_commit();
+  __syncwarp();
+  const int nk_dyn = a.topk * S * S;
+  const int nkeys = nk_dyn + a.n_fixed * (a.g.ns + a.g.Hp * a.g.Wp);
+  const int nblk = (nkeys + SEL_BN - 1) / SEL_BN;
+  auto issue = [&](int blk, int st) {
+    const uint32_t sK = sKV + st * 2 * SEL_TILE;
+    const uint32_t sV = sK + SEL_TILE;
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int e = lane + 32 * it;
+      const int key = e >> 3, c = e & 7;
+      long long off;
+      bool spec;
+      const bool ok = key_src<S>(a, sReg, blk * SEL_BN + key, nk_dyn, nkeys, off, spec);
+      const __nv_bfloat16* kp = (spec ? ksh : kh) + off * D + c * 8;
+      const __nv_bfloat16* vp = (spec ? vsh : vh) + off * D + c * 8;
+      cp_async16(sK + swz(key, c), ok ? kp : kh, ok ? 16 : 0);
+      cp_async16(sV + swz(key, c), ok ? vp : vh, ok ? 16 : 0);
+      if (c == 0) sValid[st * SEL_BN + key] = ok ? 1 : 0;
+    }
+  };
+  const float sl2 = a.scale_log2;
+  const float scale = a.scale_log2 / LOG2E;
+
+  // ---- pass 1: the forward again (online softmax), for O_sel and the row log-sum-exp
+  issue(0, 0);
+  cp_async_commit();
+  cp_async_wait<1>();
+  __syncwarp();
+  uint32_t qf[4][4];
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks)
+    ldsm_x4(sQ + swz(lr + 8 * (mi & 1), 2 * ks + (mi >> 1)), qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3]);
+  float o[8][4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+  for (int blk = 0; blk < nblk; ++blk) {
+    const int st = blk & 1;
+    __syncwarp();
+    if (blk + 1 < nblk) issue(blk + 1, st ^ 1);
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncwarp();
+    const uint32_t sK = sKV + st * 2 * SEL_TILE, sV = sK + SEL_TILE;
+    float s[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+      for (int np = 0; np < 2; ++np) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(sK + swz(16 * np + lr + 8 * (mi >> 1), 2 * ks + (mi & 1)), b0, b1, b2, b3);
+        mma_bf16(s[2 * np], qf[ks], b0, b1);
+        mma_bf16(s[2 * np + 1], qf[ks], b2, b3);
+      }
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e)
+        if (!sValid[st * SEL_BN + 8 * nt + 2 * t + e]) s[nt][e] = s[nt][2 + e] = -INFINITY;
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      float mx = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) mx = fmaxf(mx, fmaxf(s[nt][2 * rr], s[nt][2 * rr + 1]));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const float m_new = fmaxf(m[rr], mx);
+      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+      const float alpha = ex2((m[rr] - m_use) * sl2);
+      l[rr] *= alpha;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        o[nt][2 * rr] *= alpha;
+        o[nt][2 * rr + 1] *= alpha;
+      }
+      const float mb = m_use * sl2;
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
+        const float p0 = ex2(fmaf(s[nt][2 * rr], sl2, -mb));
+        const float p1 = ex2(fmaf(s[nt][2 * rr + 1], sl2, -mb));
+        s[nt][2 * rr] = p0;
+        s[nt][2 * rr + 1] = p1;
+        l[rr] += p0 + p1;
+      }
+      m[rr] = m_new;
+    }
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk) {
+      uint32_t pa[4];
+      pa[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
+      pa[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
+      pa[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+      pa[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+#pragma unroll
+      for (int dp = 0; dp < 4; ++dp) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(sV + swz(16 * kk + lr + 8 * (mi & 1), 2 * dp + (mi >> 1)), b0, b1, b2, b3);
+        mma_bf16(o[2 * dp], pa, b0, b1);
+        mma_bf16(o[2 * dp + 1], pa, b2, b3);
+      }
+    }
+  }
+  cp_async_wait<0>();
+  __syncwarp();
+
+  // ---- gate backward and the window's upsample backward --------------------------
+  bool qv[2];
+  long long tok[2];
+  float lse[2], inv[2];
+#pragma unroll
+  for (int rr = 0; rr < 2; ++rr) {
+    l[rr] += __shfl_xor_sync(0xffffffffu, l[rr], 1);
+    l[rr] += __shfl_xor_sync(0xffffffffu, l[rr], 2);
+    const int row = g + 8 * rr;
+    const int y = wi * S + row / S, x = wj * S + row % S;
+    qv[rr] = row < S * S && y < a.g.Hv && x < a.g.Wv && l[rr] > 0.f;
+    tok[rr] = (static_cast<long long>(f) * a.g.Hp + y) * a.g.Wp + x;
+    inv[rr] = qv[rr] ? 1.f / l[rr] : 0.f;
+    lse[rr] = qv[rr] ? m[rr] * sl2 + __log2f(l[rr]) : INFINITY;   // +inf: P = 0 on pad rows
+  }
+  float gg[8][4];                                   // g = sigmoid(W_g q) (or the forced gate)
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt) gg[nt][0] = gg[nt][1] = gg[nt][2] = gg[nt][3] = 0.f;
+  const __nv_bfloat16* wg = reinterpret_cast<const __nv_bfloat16*>(b.w_g) + static_cast<long long>(h) * D * D;
+  if (b.gate_mode == 0) {
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        const __nv_bfloat16* wr = wg + (8 * nt + g) * D + 16 * ks + 2 * t;
+        mma_bf16(gg[nt], qf[ks], __ldg(reinterpret_cast<const unsigned int*>(wr)),
+                 __ldg(reinterpret_cast<const unsigned int*>(wr + 8)));
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) gg[nt][e] = 1.f / (1.f + __expf(-gg[nt][e]));
+    }
+  } else {
+    const float gfix = b.gate_mode == 1 ? 1.f : 0.f;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) gg[nt][0] = gg[nt][1] = gg[nt][2] = gg[nt][3] = gfix;
+  }
+  const __nv_bfloat16* dOh = b.d_o + h * img_hs;
+  const float* ocr = b.o_comp + (static_cast<long long>(h) * a.R + r) * D;
+  float* dah = b.da + h * img_hs;
+  float Dr[2] = {0.f, 0.f};
+  float docs[8][2];                                  // column sums of g * dO over the window
+  float dq[8][4];                                    // dq_gate / scale, then + dS K
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt) {
+    const float2 oc = __ldg(reinterpret_cast<const float2*>(ocr + 8 * nt + 2 * t));
+    docs[nt][0] = docs[nt][1] = 0.f;
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      float2 dov = make_float2(0.f, 0.f);
+      if (qv[rr])
+        dov = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(dOh + tok[rr] * D + 8 * nt + 2 * t));
+      const float d0 = dov.x, d1 = dov.y;
+      const float os0 = o[nt][2 * rr] * inv[rr], os1 = o[nt][2 * rr + 1] * inv[rr];
+      const float g0 = gg[nt][2 * rr], g1 = gg[nt][2 * rr + 1];
+      const float da0 = b.gate_mode == 0 ? d0 * (oc.x - os0) * g0 * (1.f - g0) : 0.f;
+      const float da1 = b.gate_mode == 0 ? d1 * (oc.y - os1) * g1 * (1.f - g1) : 0.f;
+      docs[nt][0] += g0 * d0;
+      docs[nt][1] += g1 * d1;
+      const float dos0 = (1.f - g0) * d0, dos1 = (1.f - g1) * d1;
+      Dr[rr] += dos0 * os0 + dos1 * os1;
+      o[nt][2 * rr] = dos0;                          // o now holds dO_sel
+      o[nt][2 * rr + 1] = dos1;
+      gg[nt][2 * rr] = da0;                          // gg now holds da
+      gg[nt][2 * rr + 1] = da1;
+      const int row = g + 8 * rr;
+      if (row < S * S)
+        *reinterpret_cast<float2*>(dah + tok[rr] * D + 8 * nt + 2 * t) = make_float2(da0, da1);
+    }
+  }
+#pragma unroll
+  for (int rr = 0; rr < 2; ++rr) {
+    Dr[rr] += __shfl_xor_sync(0xffffffffu, Dr[rr], 1);
+    Dr[rr] += __shfl_xor_sync(0xffffffffu, Dr[rr], 2);
+  }
+  // dO'_comp[r] = sum over the window's valid tokens of g dO (the window is region r)
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      float v = docs[nt][e];
+      v += __shfl_xor_sync(0xffffffffu, v, 4);
+      v += __shfl_xor_sync(0xffffffffu, v, 8);
+      v += __shfl_xor_sync(0xffffffffu, v, 16);
+      docs[nt][e] = v;
+    }
+  if (g == 0) {
+    float* dst = b.d_ocomp + (static_cast<long long>(h) * a.R + r) * D;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+      *reinterpret_cast<float2*>(dst + 8 * nt + 2 * t) = make_float2(docs[nt][0], docs[nt][1]);
+  }
+  // dq from the gate: dq[k] = sum_c da[c] W_g[c][k] (B fragments from W_g's columns)
+#pragma unroll
+  for (int i = 0; i < 8; ++i) dq[i][0] = dq[i][1] = dq[i][2] = dq[i][3] = 0.f;
+  if (b.gate_mode == 0) {
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      uint32_t aa[4];
+      aa[0] = pack_bf16(gg[2 * kk][0], gg[2 * kk][1]);
+      aa[1] = pack_bf16(gg[2 * kk][2], gg[2 * kk][3]);
+      aa[2] = pack_bf16(gg[2 * kk + 1][0], gg[2 * kk + 1][1]);
+      aa[3] = pack_bf16(gg[2 * kk + 1][2], gg[2 * kk + 1][3]);
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        const int n = 8 * nt + g, k0 = 16 * kk + 2 * t;
+        const unsigned short* w16 = reinterpret_cast<const unsigned short*>(wg);
+        const uint32_t b0 = static_cast<uint32_t>(__ldg(w16 + k0 * D + n)) |
+                            (static_cast<uint32_t>(__ldg(w16 + (k0 + 1) * D + n)) << 16);
+        const uint32_t b1 = static_cast<uint32_t>(__ldg(w16 + (k0 + 8) * D + n)) |
+                            (static_cast<uint32_t>(__ldg(w16 + (k0 + 9) * D + n)) << 16);
+        mma_bf16(dq[nt], aa, b0, b1);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) dq[i][e] /= scale;
+  }
+  // dO_sel: A fragments and a swizzled bf16 tile (B operand of dV = P^T dO_sel)
+  uint32_t dof[4][4];
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+    dof[kk][0] = pack_bf16(o[2 * kk][0], o[2 * kk][1]);
+    dof[kk][1] = pack_bf16(o[2 * kk][2], o[2 * kk][3]);
+    dof[kk][2] = pack_bf16(o[2 * kk + 1][0], o[2 * kk + 1][1]);
+    dof[kk][3] = pack_bf16(o[2 * kk + 1][2], o[2 * kk + 1][3]);
+  }
+  uint8_t* sdOp = wbase + SB_DO;
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr)
+      *reinterpret_cast<uint32_t*>(sdOp + swz(g + 8 * rr, nt) + 4 * t) = pack_bf16(o[nt][2 * rr], o[nt][2 * rr + 1]);
+  __syncwarp();
+
+  // ---- pass 2: dS = P (dP - D); dq += dS K; dK += dS^T q, dV += P^T dO_sel (atomics)
+  float* dkh = b.dk + h * img_hs;
+  float* dvh = b.dv + h * img_hs;
+  float* dksh = b.dk_spec ? b.dk_spec + h * spec_hs : nullptr;
+  float* dvsh = b.dv_spec ? b.dv_spec + h * spec_hs : nullptr;
+  const uint32_t sdSt_a = smem_u32(sdSt), sPt_a = smem_u32(sPt);
+  issue(0, 0);
+  cp_async_commit();
+  for (int blk = 0; blk < nblk; ++blk) {
+    const int st = blk & 1;
+    __syncwarp();
+    if (blk + 1 < nblk) issue(blk + 1, st ^ 1);
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncwarp();
+    const uint32_t sK = sKV + st * 2 * SEL_TILE, sV = sK + SEL_TILE;
+    float s[4][4], dp[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = dp[i][0] = dp[i][1] = dp[i][2] = dp[i][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+      for (int np = 0; np < 2; ++np) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(sK + swz(16 * np + lr + 8 * (mi >> 1), 2 * ks + (mi & 1)), b0, b1, b2, b3);
+        mma_bf16(s[2 * np], qf[ks], b0, b1);
+        mma_bf16(s[2 * np + 1], qf[ks], b2, b3);
+        ldsm_x4(sV + swz(16 * np + lr + 8 * (mi >> 1), 2 * ks + (mi & 1)), b0, b1, b2, b3);
+        mma_bf16(dp[2 * np], dof[ks], b0, b1);
+        mma_bf16(dp[2 * np + 1], dof[ks], b2, b3);
+      }
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int key = 8 * nt + 2 * t + (e & 1), rr = e >> 1;
+        const float p = sValid[st * SEL_BN + key] ? ex2(fmaf(s[nt][e], sl2, -lse[rr])) : 0.f;
+        const float ds = p * (dp[nt][e] - Dr[rr]);
+        s[nt][e] = ds;
+        const int q = g + 8 * rr;
+        sdSt[key * 16 + q] = __float2bfloat16_rn(ds);      // [key][query]
+        sPt[key * 16 + q] = __float2bfloat16_rn(p);
+      }
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk) {
+      uint32_t pa[4];
+      pa[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
+      pa[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
+      pa[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+      pa[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+#pragma unroll
+      for (int dp2 = 0; dp2 < 4; ++dp2) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(sK + swz(16 * kk + lr + 8 * (mi & 1), 2 * dp2 + (mi >> 1)), b0, b1, b2, b3);
+        mma_bf16(dq[2 * dp2], pa, b0, b1);
+        mma_bf16(dq[2 * dp2 + 1], pa, b2, b3);
+      }
+    }
+    __syncwarp();
+    // dK and dV of the block's 32 keys, 16 at a time, straight to global memory
+#pragma unroll 1
+    for (int half = 0; half < 4; ++half) {
+      const int mt = half & 1;
+      const bool isv = half >= 2;
+      uint32_t af[4];
+      ldsm_pitch32(isv ? sPt_a : sdSt_a, 16 * mt, af);
+      float acc[8][4];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+#pragma unroll
+      for (int dp2 = 0; dp2 < 4; ++dp2) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t((isv ? sdO : sQ) + swz(lr + 8 * (mi & 1), 2 * dp2 + (mi >> 1)), b0, b1, b2, b3);
+        mma_bf16(acc[2 * dp2], af, b0, b1);
+        mma_bf16(acc[2 * dp2 + 1], af, b2, b3);
+      }
+      const float mul = isv ? 1.f : scale;
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        const int key = 16 * mt + g + 8 * rr;
+        if (!sValid[st * SEL_BN + key]) continue;
+        long long off;
+        bool spec;
+        key_src<S>(a, sReg, blk * SEL_BN + key, nk_dyn, nkeys, off, spec);
+        float* base = spec ? (isv ? dvsh : dksh) : (isv ? dvh : dkh);
+        if (!base) continue;
+        base += off * D + 2 * t;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+          atomicAdd(reinterpret_cast<float2*>(base + 8 * nt), make_float2(acc[nt][2 * rr] * mul, acc[nt][2 * rr + 1] * mul));
+      }
+    }
+  }
+  cp_async_wait<0>();
+  // dq of the window's tokens: scale (dS K + dq_gate / scale); pad rows 0
+  float* dqh = b.dq + h * img_hs;
+#pragma unroll
+  for (int rr = 0; rr < 2; ++rr) {
+    const int row = g + 8 * rr;
+    if (row >= S * S) continue;
+    const int y = wi * S + row / S, x = wj * S + row % S;
+    const bool valid = y < a.g.Hv && x < a.g.Wv;
+    const long long tk = (static_cast<long long>(f) * a.g.Hp + y) * a.g.Wp + x;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+      *reinterpret_cast<float2*>(dqh + tk * D + 8 * nt + 2 * t) =
+          valid ? make_float2(dq[nt][2 * rr] * scale, dq[nt][2 * rr + 1] * scale) : make_float2(0.f, 0.f);
+  }
+}
+
+template <int S>
+cudaError_t launch_sel_bwd_s(const SelBwdArgs& b, cudaStream_t st) {
+  const int sm = SEL_WARPS * SB_WARP;
+  cudaError_t e = cudaFuncSetAttribute(sel_bwd_kernel<S>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+  if (e != cudaSuccess) return e;
+  const long long w = static_cast<long long>(b.s.H) * b.s.R;
+  sel_bwd_kernel<S><<<static_cast<unsigned>((w + SEL_WARPS - 1) / SEL_WARPS), SEL_WARPS * 32, sm, st>>>(b);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_sel_bwd(const SelBwdArgs& b, cudaStream_t st) {
+  switch (b.s.s) {
+    case 1: return launch_sel_bwd_s<1>(b, st);
+    case 2: return launch_sel_bwd_s<2>(b, st);
+    case 4: return launch_sel_bwd_s<4>(b, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace gsa
