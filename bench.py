@@ -434,6 +434,42 @@ def run_b200(args, cfg, rank, world, local, dist):
                           f"{r['spec_rows']} special rows, {r['sample_s']:.1f} s of CPU work, extrapolated to "
                           f"all windows and heads; BLAS {blas}; {cores} cores visible")}
 
+    # ---- backward pass (optional): gradients of every input, selection held fixed ----
+    backward = None
+    if args.backward:
+        dout = {k: (torch.randn(v.shape, device=dev) * 0.5).to(v.dtype) for k, v in out.items()}
+        fwd = layer.forward(x, out=out)
+        for _ in range(2):
+            gr = layer.backward(x, fwd, dout)
+        torch.cuda.synchronize()
+        barrier()
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b0.record(stream)
+        for _ in range(3):
+            gr = layer.backward(x, fwd, dout)
+        b1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        bms = max_over_ranks(b0.elapsed_time(b1) / 3, dist, dev)
+        gsa.gsa_set_profiling(layer.ctx, True)
+        gr = layer.backward(x, fwd, dout)
+        bk = {n: round(t, 3) for n, t in gsa.gsa_get_kernel_times(layer.ctx)}
+        gsa.gsa_set_profiling(layer.ctx, False)
+        st = layer.status()
+        if st != 0:
+            raise RuntimeError(f"device status {st} in the backward: {gsa.gsa_strerror(st)}")
+        d = cfg.head_dim
+        H = cfg.num_heads
+        fl = {"bwd_comp_attn": 10.0 * d * cfg.num_regions ** 2 * H,
+              "bwd_selection_gate": 10.0 * d * cfg.num_img_valid * cfg.topk * cfg.pool_s ** 2 * H,
+              "bwd_special": 10.0 * d * cfg.num_spec * (cfg.num_spec + cfg.num_img_valid) * H}
+        kern = {n: ({"ms": t, "tflops": round(fl[n] / (t / 1e3) / 1e12, 1)} if n in fl else {"ms": t})
+                for n, t in bk.items()}
+        backward = {"ms": round(bms, 3), "vs_forward": round(bms / ms, 2),
+                    "flops_convention": "10*d per (query, key) pair and attention (S, dP, dQ, dK, dV)",
+                    "kernels": kern}
+        del gr, dout
+
     layer.close()
 
     # ---- ablation variants of the notes' table, same inputs (optional) -------------
@@ -496,6 +532,8 @@ def run_b200(args, cfg, rank, world, local, dist):
     }
     if ablations is not None:
         line["ablations"] = ablations
+    if backward is not None:
+        line["backward"] = backward
     return line
 
 
@@ -509,6 +547,8 @@ def main():
     ap.add_argument("--dense", default="full", choices=["full", "off"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="also time gsa_backward (gradients of every input) on the same inputs")
     ap.add_argument("--ablations", action="store_true",
                     help="also time the layer variants of the ablation table (no compressed value, "
                          "no selection, top-8/16/64) on the same inputs")

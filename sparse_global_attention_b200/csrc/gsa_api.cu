@@ -694,6 +694,7 @@ int gsa_backward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void*
   if (!k_spec) k_spec = k_img;
   if (!v_spec) v_spec = v_img;
   if (!w_g) w_g = q_img;
+  Prof prof(c, st);
   // gradients reached by atomics or accumulation start at zero
   if (cudaMemsetAsync(dk_img, 0, img * D * 4, st) != cudaSuccess || cudaMemsetAsync(dv_img, 0, img * D * 4, st) != cudaSuccess)
     return GSA_ERR_CUDA;
@@ -716,6 +717,7 @@ int gsa_backward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void*
   sb.dk_spec = spec ? dk_spec : nullptr; sb.dv_spec = spec ? dv_spec : nullptr;
   sb.d_ocomp = docomp; sb.da = da;
   if (launch_sel_bwd(sb, st) != cudaSuccess) return GSA_ERR_CUDA;
+  prof.mark("bwd_selection_gate");
 
   // 2. compressed attention (split guide scores, as in the forward)
   const long long rhs = static_cast<long long>(d.R) * D;
@@ -733,6 +735,7 @@ int gsa_backward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void*
   ba.dk[0] = dkc; ba.dv[0] = dvc; ba.dkv_hs[0] = rhs; ba.dkv_accum = 0;
   ba.H = H; ba.g = g; ba.scale_log2 = scale * LOG2E; ba.scale = scale;
   if (launch_attn_bwd(ba, st) != cudaSuccess) return GSA_ERR_CUDA;
+  prof.mark("bwd_comp_attn");
 
   // 3. pooling: each valid token takes its region's gradient over the region's size
   PoolBwdArgs pb;
@@ -741,6 +744,7 @@ int gsa_backward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void*
   pb.H = H; pb.F = cf.num_frames; pb.Hp = cf.pad_h; pb.Wp = cf.pad_w; pb.Hv = cf.grid_h; pb.Wv = cf.grid_w;
   pb.s = cf.pool_s;
   if (launch_pool_bwd(pb, st) != cudaSuccess) return GSA_ERR_CUDA;
+  prof.mark("bwd_pool");
 
   // 4. special tokens over every special and valid image token
   if (spec) {
@@ -764,6 +768,7 @@ int gsa_backward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void*
     bs.dk[1] = dk_img; bs.dv[1] = dv_img; bs.dkv_hs[1] = ihs; bs.dkv_accum = 1;
     bs.H = H; bs.g = g; bs.scale_log2 = scale * LOG2E; bs.scale = scale;
     if (launch_attn_bwd(bs, st) != cudaSuccess) return GSA_ERR_CUDA;
+    prof.mark("bwd_special");
   }
 
   // 5. the gate matrix
@@ -773,6 +778,7 @@ int gsa_backward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void*
   } else if (cudaMemsetAsync(dw_g, 0, static_cast<size_t>(H) * D * D * 4, st) != cudaSuccess) {
     return GSA_ERR_CUDA;
   }
+  prof.mark("bwd_gate_weight");
   return GSA_OK;
 }
 
