@@ -19,9 +19,13 @@ NO_SPECIAL_BF16 = GSAConfig("no_special_bf16", 4, 16, 16, 16, 16, 0, 1, 64, 4, 5
 PAD_F32 = GSAConfig("pad_vggt_f32", 4, 7, 7, 8, 8, 2, 2, 64, 2, 5, "fp32", (1,))
 S8_BF16 = GSAConfig("s8_bf16", 3, 16, 16, 16, 16, 2, 2, 64, 8, 3, "bf16")                  # 8x8 windows, R=12
 S8_PAD_BF16 = GSAConfig("s8_pad_bf16", 2, 14, 13, 16, 16, 1, 2, 64, 8, 2, "bf16")          # ragged 8x8 windows
+# degenerate shapes: s = 1 (pooling is the identity), one frame, k = 1, one head
+S1_BF16 = GSAConfig("s1_bf16", 2, 6, 7, 6, 7, 1, 2, 64, 1, 5, "bf16")                       # R = 84 tokens
+ONE_FRAME_BF16 = GSAConfig("one_frame_bf16", 1, 12, 12, 12, 12, 3, 1, 64, 4, 3, "bf16")
+TOPK1_BF16 = GSAConfig("topk1_bf16", 4, 8, 8, 8, 8, 1, 2, 64, 2, 1, "bf16")
 
 SMALL = [CONFIGS["tiny_fp32"], RAGGED_BF16, MULTI_TILE_BF16, S2_BF16, PAD_VGGT_BF16,
-         NO_SPECIAL_BF16, PAD_F32, S8_BF16, S8_PAD_BF16]
+         NO_SPECIAL_BF16, PAD_F32, S8_BF16, S8_PAD_BF16, S1_BF16, ONE_FRAME_BF16, TOPK1_BF16]
 
 
 def _cuda_inputs(cfg, seed=0):
@@ -82,6 +86,19 @@ def test_pi3_32_frames_parity():
         tot_checked += c
         tot_under += u
     assert tot_checked > 0
+
+
+@pytest.mark.parametrize("k", [64, 16, 8])
+def test_pi3_32_frames_other_topk(k):
+    """The list lengths of the ablation (top-8/16/64): the register-list kernels for k = 8, 16, 64."""
+    cfg = CONFIGS["pi3_f32"].with_(topk=k)
+    x = _cuda_inputs(cfg)
+    res = run_gpu(cfg, x)
+    checked = 0
+    for h in (0, 15):
+        c, _ = compare_head(cfg, x, res, h)
+        checked += c
+    assert checked > 0
 
 
 def _sample_windows(cfg, n, seed):
