@@ -154,21 +154,31 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) sel_kernel_bf16(const SelArgs 
   const int nkeys = nk_dyn + a.n_fixed * (a.g.ns + a.g.Hp * a.g.Wp);
   const int nblk = (nkeys + SEL_BN - 1) / SEL_BN;
 
+  // each lane resolves one key of the block (the warp's 32, or 8 with s = 8)
+  // and hands its source to the 8 lanes that copy that key's 128-byte row:
+  // src >= 0 image token, src <= -2 special token -(src + 2), -1 no key
   auto issue = [&](int blk, int st) {
     const uint32_t sK = sKVs + st * 2 * SEL_TILE;
     const uint32_t sV = sK + SEL_TILE;
-#pragma unroll
-    for (int it = 0; it < (SH ? 2 : 8); ++it) {
-      const int e = lane + 32 * it;
-      const int key = (SH ? 8 * warp : 0) + (e >> 3), c = e & 7;
+    constexpr int NKW = SH ? 8 : 32;              // keys this warp copies per block
+    const int kbase = SH ? 8 * warp : 0;
+    long long mine = -1;
+    if (lane < NKW) {
       long long off;
       bool spec;
-      const bool ok = key_src<S>(a, sReg, blk * SEL_BN + key, nk_dyn, nkeys, off, spec);
-      const __nv_bfloat16* kp = (spec ? ksh : kh) + off * D + c * 8;
-      const __nv_bfloat16* vp = (spec ? vsh : vh) + off * D + c * 8;
-      cp_async16(sK + swz(key, c), ok ? kp : kh, ok ? 16 : 0);
-      cp_async16(sV + swz(key, c), ok ? vp : vh, ok ? 16 : 0);
-      if (c == 0) sValidS[st * SEL_BN + key] = ok ? 1 : 0;
+      if (key_src<S>(a, sReg, blk * SEL_BN + kbase + lane, nk_dyn, nkeys, off, spec)) mine = spec ? -(off + 2) : off;
+      sValidS[st * SEL_BN + kbase + lane] = mine != -1 ? 1 : 0;
+    }
+#pragma unroll
+    for (int it = 0; it < NKW / 4; ++it) {
+      const int local = (lane >> 3) + 4 * it, c = lane & 7;
+      const long long src = __shfl_sync(0xffffffffu, mine, local);
+      const bool ok = src != -1;
+      const bool spec = src <= -2;
+      const long long off = spec ? -(src + 2) : (ok ? src : 0);
+      const int key = kbase + local;
+      cp_async16(sK + swz(key, c), (spec ? ksh : kh) + off * D + c * 8, ok ? 16 : 0);
+      cp_async16(sV + swz(key, c), (spec ? vsh : vh) + off * D + c * 8, ok ? 16 : 0);
     }
   };
 
@@ -513,21 +523,25 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) sel_bwd_kernel(const SelBwdArg
   const int nk_dyn = a.topk * S * S;
   const int nkeys = nk_dyn + a.n_fixed * (a.g.ns + a.g.Hp * a.g.Wp);
   const int nblk = (nkeys + SEL_BN - 1) / SEL_BN;
-  auto issue = [&](int blk, int st) {
+  auto issue = [&](int blk, int st) {               // one key per lane, rows copied by 8 lanes
     const uint32_t sK = sKV + st * 2 * SEL_TILE;
     const uint32_t sV = sK + SEL_TILE;
-#pragma unroll
-    for (int it = 0; it < 8; ++it) {
-      const int e = lane + 32 * it;
-      const int key = e >> 3, c = e & 7;
+    long long mine = -1;
+    {
       long long off;
       bool spec;
-      const bool ok = key_src<S>(a, sReg, blk * SEL_BN + key, nk_dyn, nkeys, off, spec);
-      const __nv_bfloat16* kp = (spec ? ksh : kh) + off * D + c * 8;
-      const __nv_bfloat16* vp = (spec ? vsh : vh) + off * D + c * 8;
-      cp_async16(sK + swz(key, c), ok ? kp : kh, ok ? 16 : 0);
-      cp_async16(sV + swz(key, c), ok ? vp : vh, ok ? 16 : 0);
-      if (c == 0) sValid[st * SEL_BN + key] = ok ? 1 : 0;
+      if (key_src<S>(a, sReg, blk * SEL_BN + lane, nk_dyn, nkeys, off, spec)) mine = spec ? -(off + 2) : off;
+      sValid[st * SEL_BN + lane] = mine != -1 ? 1 : 0;
+    }
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int key = (lane >> 3) + 4 * it, c = lane & 7;
+      const long long src = __shfl_sync(0xffffffffu, mine, key);
+      const bool ok = src != -1;
+      const bool spec = src <= -2;
+      const long long off = spec ? -(src + 2) : (ok ? src : 0);
+      cp_async16(sK + swz(key, c), (spec ? ksh : kh) + off * D + c * 8, ok ? 16 : 0);
+      cp_async16(sV + swz(key, c), (spec ? vsh : vh) + off * D + c * 8, ok ? 16 : 0);
     }
   };
   const float sl2 = a.scale_log2;
