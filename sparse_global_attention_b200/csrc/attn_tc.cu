@@ -16,10 +16,13 @@
 //              read from TMEM, V as an MN-major shared-memory operand)
 // TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,320), O_1 [320,384),
 // P_0 [384,448), P_1 [448,512) (bf16 pairs).
-// Softmax threads read their row of S_i, write P_i (bf16 pairs) back over the
-// first 64 columns of S_i, and rescale O_i in TMEM only when the running max
-// grows by more than 2^8 (lazy rescaling: the stale max keeps every
-// exponent <= 2^8, and numerator and denominator share it).
+// Softmax threads read their row of S_i, write P_i (bf16 pairs) to its own
+// TMEM columns, and rescale O_i in TMEM only when the running max grows by
+// more than 2^8 (lazy rescaling: the stale max keeps every exponent <= 2^8,
+// and numerator and denominator share it).  The two softmax warpgroups run
+// their exponentials at the same time: with two warps per SM sub-partition
+// feeding the MUFU, one warp's non-MUFU instructions and dependency stalls
+// are covered by the other's exponentials.
 //
 // Guide scores (K2): Q and K arrive as bf16 pairs hi + lo (lo = bf16 of the
 // residual), S = Qhi Khi^T + Qhi Klo^T + Qlo Khi^T, accurate to ~2^-17 of
@@ -63,9 +66,8 @@ struct Lay {
   static constexpr int KV = 2 * QT * TILE;             // Q_i hi at i*TILE, lo at (2+i)*TILE
   static constexpr int STAGE = KT * TILE;
   static constexpr int BAR = KV + NST * STAGE;
-  // barriers: q_full, full[NST], empty[NST], s_full[2], s_free[2], p_full[2], pv_done[2], fin,
-  // turn[2]
-  static constexpr int NBAR = 1 + 2 * NST + 8 + 1 + 2;
+  // barriers: q_full, full[NST], empty[NST], s_full[2], s_free[2], p_full[2], pv_done[2], fin
+  static constexpr int NBAR = 1 + 2 * NST + 8 + 1;
   static constexpr int TMEM_SLOT = BAR + NBAR * 8;
   static constexpr int BYTES = TMEM_SLOT + 16 + 1024;   // + alignment slack
 };
@@ -81,23 +83,12 @@ struct Bars {
   __device__ uint32_t p_full(int i) const { return base + 8 * (5 + 2 * nst + i); }
   __device__ uint32_t pv_done(int i) const { return base + 8 * (7 + 2 * nst + i); }
   __device__ uint32_t fin() const { return base + 8 * (9 + 2 * nst); }
-  __device__ uint32_t turn(int i) const { return base + 8 * (10 + 2 * nst + i); }
 };
 
 // one arrival per warp, after every lane's preceding work (fences included)
 __device__ __forceinline__ void warp_arrive(uint32_t bar) {
   __syncwarp();
   if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
-}
-
-// The two softmax warpgroups take turns on their exponential phase (the MUFU
-// work of a tile): warpgroup 0 runs tile j after warpgroup 1 finished tile
-// j-1, warpgroup 1 runs tile j after warpgroup 0 finished tile j, so one
-// group's exponentials overlap the other's loads, maxima and waits.
-__device__ __forceinline__ bool exp_turn_wait(const Bars& bars, int qi, int j, int* err) {
-  if (qi == 0 && j == 0) return true;
-  const uint32_t par = static_cast<uint32_t>(qi == 0 ? (j - 1) : j) & 1u;
-  return __all_sync(0xffffffffu, mbar_wait(bars.turn(qi), par, err));
 }
 
 __device__ __forceinline__ int tile_seg(const AttnArgs& a, int tt, long long& kb) {
@@ -307,7 +298,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(bars.s_free(i), TBM / 32);     // one arrival per softmax warp
       mbar_init(bars.p_full(i), TBM / 32);
       mbar_init(bars.pv_done(i), 1);
-      mbar_init(bars.turn(i), TBM / 32);
     }
     mbar_init(bars.fin(), 1);
     fence_mbar_init();
@@ -483,8 +473,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           ok = __all_sync(0xffffffffu, mbar_wait(bars.pv_done(qi), (j - 1) & 1, a.err));
           if (!ok) break;
         }
-        ok = exp_turn_wait(bars, qi, j, a.err);
-        if (!ok) break;
         const float mb = (m == -INFINITY) ? 0.f : m * sl2;
         float l0 = 0.f, l1 = 0.f;
 #pragma unroll
@@ -498,7 +486,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
           tmem_st16(tP + 16 * c, pk);
         }
-        warp_arrive(bars.turn(qi ^ 1));
         l += l0 + l1;
       } else {
         // pass 1, two 64-key halves: row max and the streaming top-k
@@ -553,8 +540,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           ok = __all_sync(0xffffffffu, mbar_wait(bars.pv_done(qi), (j - 1) & 1, a.err));
           if (!ok) break;
         }
-        ok = exp_turn_wait(bars, qi, j, a.err);
-        if (!ok) break;
         const float mb = (m == -INFINITY) ? 0.f : m * sl2;
         float l0 = 0.f, l1 = 0.f;
 #pragma unroll 1
@@ -578,7 +563,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
           tmem_st32(tP + 32 * hf, pk);
         }
-        warp_arrive(bars.turn(qi ^ 1));
         l += l0 + l1;
       }
       tmem_wait_st();          // P (and any O rescale) written to TMEM
