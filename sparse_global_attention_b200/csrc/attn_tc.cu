@@ -221,6 +221,7 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
 // Lazy rescale: move the reference max only when the row max grew by more than
 // 2^8; O_i (in TMEM) is rescaled once PV of the previous tile has completed.
 // The decision to touch TMEM is warp-uniform (TMEM loads are warp-collective).
+template <int PIECE>
 __device__ __forceinline__ void rescale(float mx, float& m, float& l, int j, int qi, uint32_t tO,
                                         const Bars& bars, int* err, bool& ok, float sl2) {
   const float m_new = fmaxf(m, mx);
@@ -235,17 +236,40 @@ __device__ __forceinline__ void rescale(float mx, float& m, float& l, int j, int
     ok = __all_sync(0xffffffffu, mbar_wait(bars.pv_done(qi), (j - 1) & 1, err));
     if (!ok) return;
     tc_fence_after();
+    if constexpr (PIECE == 8) {
+      // eight columns at a time: the caller holds a half-row of S and its top-k list
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {
+        uint32_t w[8];
+        tmem_ld8(tO + 8 * c, w);
+        tmem_wait_ld();
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      uint32_t v[32];
-      tmem_ld32(tO + 32 * c, v);
-      tmem_wait_ld();
+        for (int e = 0; e < 8; ++e) w[e] = __float_as_uint(__uint_as_float(w[e]) * alpha);
+        tmem_st8(tO + 8 * c, w);
+      }
+    } else {
 #pragma unroll
-      for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-      tmem_st32(tO + 32 * c, v);
+      for (int c = 0; c < 2; ++c) {
+        uint32_t w[32];
+        tmem_ld32(tO + 32 * c, w);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) w[e] = __float_as_uint(__uint_as_float(w[e]) * alpha);
+        tmem_st32(tO + 32 * c, w);
+      }
     }
     tmem_wait_st();
   }
+}
+
+// current k-th score of the list (the list may be longer than the run's k)
+template <int KC>
+__device__ __forceinline__ float kth_score(const float (&ts)[KC > 0 ? KC : 1], int kc) {
+  if (kc == KC) return ts[KC - 1];
+  uint32_t t = __float_as_uint(ts[KC - 1]);
+#pragma unroll
+  for (int p = 0; p < KC; ++p) t = sel_if(p == kc - 1, __float_as_uint(ts[p]), t);
+  return __uint_as_float(t);
 }
 
 template <int KC>
@@ -466,7 +490,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           cm[c] = max32(v + 32 * c);
         }
         mx = fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3]));
-        rescale(mx, m, l, j, qi, tO, bars, a.err, ok, sl2);
+        rescale<32>(mx, m, l, j, qi, tO, bars, a.err, ok, sl2);
         if (!ok) break;
         // P_i is free once PV of the previous tile has completed
         if (j > 0) {
@@ -488,19 +512,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         l += l0 + l1;
       } else {
-        // pass 1, two 64-key halves: row max and the streaming top-k
+        // One pass over two 64-key halves.  Each half: row max and the streaming
+        // top-k, then (unless guide only) its part of the online softmax, so S_i
+        // is read once and handed back to the MMA warp as soon as its second
+        // half is in registers: S_{i,j+1} then overlaps most of this tile.
+        float l0 = 0.f, l1 = 0.f;
 #pragma unroll 1
         for (int hf = 0; hf < 2; ++hf) {
           uint32_t v[64];
           tmem_ld64(tS + 64 * hf, v);
           tmem_wait_ld();
+          if (hf == 1) {
+            tc_fence_before();
+            warp_arrive(bars.s_free(qi));
+          }
           uint32_t cb[2] = {0u, 0u};
+          float hmx = -INFINITY;
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             const uint32_t msk = sel_if(hf, vm[2 + c], vm[c]);
             if (msk != ~0u) apply_mask(v + 32 * c, msk);
             const float cmax = max32(v + 32 * c);
-            mx = fmaxf(mx, cmax);
+            hmx = fmaxf(hmx, cmax);
             if (cmax > thr) {
 #pragma unroll
               for (int e = 0; e < 32; ++e) cb[c] |= (__uint_as_float(v[32 * c + e]) > thr ? 1u : 0u) << e;
@@ -516,53 +549,54 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int col = static_cast<int>(kb) + 64 * hf + e;
             if (!(x > thr) || (a.n_fixed && is_fixed_region(a, col))) continue;
             topk_insert<KC>(ts, ti, x, col);
-            if (a.kc == KC) {
-              thr = ts[KC - 1];
-            } else {
-              uint32_t t = __float_as_uint(ts[KC - 1]);
-#pragma unroll
-              for (int p = 0; p < KC; ++p) t = sel_if(p == a.kc - 1, __float_as_uint(ts[p]), t);
-              thr = __uint_as_float(t);
-            }
+            thr = kth_score<KC>(ts, a.kc);
           }
-        }
-        if constexpr (GO) {
-          // guide only: S_i goes straight back, nothing else to compute
-          tc_fence_before();
-          warp_arrive(bars.s_free(qi));
-          continue;
-        }
-        rescale(mx, m, l, j, qi, tO, bars, a.err, ok, sl2);
-        if (!ok) break;
-        // pass 2: P = exp2((S - m) * scale * log2e) in bf16 to shared memory; S_i
-        // goes back to the MMA warp after its last half is read
-        if (j > 0) {
-          ok = __all_sync(0xffffffffu, mbar_wait(bars.pv_done(qi), (j - 1) & 1, a.err));
-          if (!ok) break;
-        }
-        const float mb = (m == -INFINITY) ? 0.f : m * sl2;
-        float l0 = 0.f, l1 = 0.f;
+          if constexpr (!GO) {
+            // online softmax per half: the reference max moves only when this
+            // half raises a row's max by more than 2^8 (rare after the first tile)
+            const bool grow = (m == -INFINITY) ? (hmx != -INFINITY) : ((hmx - m) * sl2 > RESCALE_LOG2);
+            if (__any_sync(0xffffffffu, grow)) {
+              l += l0 + l1;
+              l0 = l1 = 0.f;
+              const float m_old = m;
+              rescale<8>(hmx, m, l, j, qi, tO, bars, a.err, ok, sl2);
+              if (!ok) break;
+              if (hf == 1) {
+                // P of the first half was written against the old max: scale it too
+                const float alpha = (m == m_old) ? 1.f : (m_old == -INFINITY ? 0.f : ex2((m_old - m) * sl2));
+                tmem_wait_st();
 #pragma unroll 1
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t v[64];
-          tmem_ld64(tS + 64 * hf, v);
-          tmem_wait_ld();
-          if (hf == 1) {
-            tc_fence_before();
-            warp_arrive(bars.s_free(qi));
-          }
-          const uint32_t m0 = sel_if(hf, vm[2], vm[0]), m1 = sel_if(hf, vm[3], vm[1]);
-          if (m0 != ~0u) apply_mask(v, m0);
-          if (m1 != ~0u) apply_mask(v + 32, m1);
-          uint32_t pk[32];
+                for (int q = 0; q < 4; ++q) {
+                  uint32_t w[8];
+                  tmem_ld8(tP + 8 * q, w);
+                  tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 64; e += 2) {
-            float p0, p1;
-            exp2_pair(v[e], v[e + 1], sl2, -mb, l0, l1, p0, p1);
-            pk[e >> 1] = pack_bf16(p0, p1);
+                  for (int e = 0; e < 8; ++e) {
+                    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&w[e]);
+                    w[e] = pack_bf16(__low2float(b) * alpha, __high2float(b) * alpha);
+                  }
+                  tmem_st8(tP + 8 * q, w);
+                }
+              }
+            }
+            // P_i is free once PV of the previous tile has completed
+            if (hf == 0 && j > 0) {
+              ok = __all_sync(0xffffffffu, mbar_wait(bars.pv_done(qi), (j - 1) & 1, a.err));
+              if (!ok) break;
+            }
+            const float mb = (m == -INFINITY) ? 0.f : m * sl2;
+            uint32_t pk[32];
+#pragma unroll
+            for (int e = 0; e < 64; e += 2) {
+              float p0, p1;
+              exp2_pair(v[e], v[e + 1], sl2, -mb, l0, l1, p0, p1);
+              pk[e >> 1] = pack_bf16(p0, p1);
+            }
+            tmem_st32(tP + 32 * hf, pk);
           }
-          tmem_st32(tP + 32 * hf, pk);
         }
+        if (!ok) break;
+        if constexpr (GO) continue;      // guide only: nothing else to compute
         l += l0 + l1;
       }
       tmem_wait_st();          // P (and any O rescale) written to TMEM
