@@ -181,3 +181,34 @@ def test_repeated_forward_is_deterministic():
     b = run_gpu(cfg, x)
     assert torch.equal(a["o_img"], b["o_img"]) and torch.equal(a["idx"], b["idx"])
     assert torch.equal(a["o_spec"], b["o_spec"])
+
+
+def test_max_jump_inside_a_key_tile():
+    """Keys scaled up in the second 64-key half of a key tile: the compressed
+    branch's reference max moves inside the tile, so O is rescaled in TMEM and
+    the P of the first half, already written with the old max, is scaled too
+    (tile 0: no O yet; tile 1: both).  The special-token rows see the same jumps
+    through their tile-level lazy rescale."""
+    cfg = MULTI_TILE_BF16                      # 6x6 regions per frame, R = 216: two key tiles
+    x = make_inputs(cfg, seed=0)
+    k = x["k_img"].float()
+    k[:, 2] *= 6.0                             # frame 2 = regions 72..107: second half of key tile 0
+    k[:, 5, 8:] *= 14.0                        # frame 5, region rows >= 2 = regions 192..215: tile 1, second half
+    x["k_img"] = k.to(x["k_img"].dtype)
+    # the peaked softmax carries single value rows to the output; smaller values keep
+    # the bf16 output rounding inside the absolute bar (the softmax paths are unchanged)
+    for name in ("v_img", "v_spec"):
+        x[name] = (x[name].float() * 0.25).to(x[name].dtype)
+    # the construction does what it says: for a fifth or more of the compressed rows
+    # (so in practically every warp of 32 rows) the max of the scaled half exceeds
+    # everything before it by more than 2^8 (in exp2 units)
+    sl2 = np.log2(np.e) / np.sqrt(cfg.head_dim)
+    qc = oracle.pool(to_f64_numpy(x["q_img"][0]), cfg.grid_h, cfg.grid_w, cfg.pool_s).reshape(-1, 64)
+    kc = oracle.pool(to_f64_numpy(x["k_img"][0]), cfg.grid_h, cfg.grid_w, cfg.pool_s).reshape(-1, 64)
+    s = qc @ kc.T * sl2
+    assert np.mean(s[:, 64:128].max(1) - s[:, :64].max(1) > 8) > 0.18
+    assert np.mean(s[:, 192:].max(1) - s[:, :192].max(1) > 8) > 0.18
+    x = {kk: v.cuda() for kk, v in x.items()}
+    res = run_gpu(cfg, x)
+    for h in range(cfg.num_heads):
+        compare_head(cfg, x, res, h)
