@@ -528,11 +528,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
           uint32_t cb[2] = {0u, 0u};
           float hmx = -INFINITY;
+          float cmx[2];
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             const uint32_t msk = sel_if(hf, vm[2 + c], vm[c]);
             if (msk != ~0u) apply_mask(v + 32 * c, msk);
             const float cmax = max32(v + 32 * c);
+            cmx[c] = cmax;
             hmx = fmaxf(hmx, cmax);
             if (cmax > thr) {
 #pragma unroll
@@ -540,12 +542,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
           }
           // rare: a score beats the current k-th; take the candidates in column
-          // order through one insertion site for the whole half
+          // order through one insertion site for the whole half.  A chunk with a
+          // single candidate needs no select tree: the candidate is the chunk max.
+          const bool one0 = __popc(cb[0]) == 1, one1 = __popc(cb[1]) == 1;
           while (cb[0] | cb[1]) {
             const bool lo = cb[0] != 0;
             const int e = lo ? __ffs(cb[0]) - 1 : 31 + __ffs(cb[1]);
             if (lo) cb[0] &= cb[0] - 1; else cb[1] &= cb[1] - 1;
-            const float x = __uint_as_float(pick64(v, e));
+            const float x = (lo ? one0 : one1) ? (lo ? cmx[0] : cmx[1]) : __uint_as_float(pick64(v, e));
             const int col = static_cast<int>(kb) + 64 * hf + e;
             if (!(x > thr) || (a.n_fixed && is_fixed_region(a, col))) continue;
             topk_insert<KC>(ts, ti, x, col);
