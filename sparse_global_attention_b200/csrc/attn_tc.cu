@@ -717,6 +717,301 @@ cudaError_t launch_kc2(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t 
   return a.guide_only ? launch_kc<KC, true>(a, maps, st) : launch_kc<KC, false>(a, maps, st);
 }
 
+// ==== attention backward on tcgen05: dQ ======================================
+// Per CTA one 128-row query tile (thread = row = TMEM lane) against every key
+// tile: S = Q K^T (the forward's split guide where it had one) and
+// dP = dO V^T into TMEM, the softmax warps turn them into
+// dS = P o (dP - D) with P = exp2(S * scale * log2 e - lse2) (bf16 pairs into
+// TMEM), and dQ += dS K runs in the TS form with K as an MN-major operand.
+// TMEM: S [0,128), dP [128,256), dQ [256,320), dS [320,384).
+// Warps 0-3 softmax, warp 4 TMA producer, warp 5 MMA issuer.
+constexpr int BW_NTHREADS = 192;
+
+struct BwdTc {
+  BwdArgs b;
+  int tiles0;                  // 128-key tiles of segment 0
+  int tiles_total;
+  int* err;
+};
+
+template <bool SPLIT>
+struct DqLay {
+  static constexpr int NST = 3;
+  static constexpr int QT = SPLIT ? 3 : 2;     // Q hi, [Q lo], dO
+  static constexpr int KT = SPLIT ? 3 : 2;     // K hi, [K lo], V
+  static constexpr int KV = QT * TILE;
+  static constexpr int STAGE = KT * TILE;
+  static constexpr int BAR = KV + NST * STAGE;
+  // q_full, full[NST], empty[NST], s_full, s_free, ds_full, dq_done, fin
+  static constexpr int NBAR = 1 + 2 * NST + 5;
+  static constexpr int TMEM_SLOT = BAR + NBAR * 8;
+  static constexpr int BYTES = TMEM_SLOT + 16 + 1024;
+};
+
+struct DqBars {
+  uint32_t base;
+  int nst;
+  __device__ uint32_t q_full() const { return base; }
+  __device__ uint32_t full(int s) const { return base + 8 * (1 + s); }
+  __device__ uint32_t empty(int s) const { return base + 8 * (1 + nst + s); }
+  __device__ uint32_t s_full() const { return base + 8 * (1 + 2 * nst); }
+  __device__ uint32_t s_free() const { return base + 8 * (2 + 2 * nst); }
+  __device__ uint32_t ds_full() const { return base + 8 * (3 + 2 * nst); }
+  __device__ uint32_t dq_done() const { return base + 8 * (4 + 2 * nst); }
+  __device__ uint32_t fin() const { return base + 8 * (5 + 2 * nst); }
+};
+
+__device__ __forceinline__ int bw_seg(const BwdTc& t, int tt, long long& kb) {
+  const int seg = (t.b.nseg > 1 && tt >= t.tiles0) ? 1 : 0;
+  kb = static_cast<long long>(seg ? tt - t.tiles0 : tt) * TBN;
+  return seg;
+}
+
+// dS of two keys: P = exp2(s * sl2 - lse2) (packed FFMA2), dS = P (dP - D)
+__device__ __forceinline__ uint32_t ds_pair(uint32_t s0, uint32_t s1, uint32_t dp0, uint32_t dp1, float sl2,
+                                            float nlse, float nD) {
+  float x0, x1;
+  asm("{\n .reg .b64 a, b, c, d;\n"
+      " mov.b64 a, {%2, %3};\n mov.b64 b, {%4, %4};\n mov.b64 c, {%5, %5};\n"
+      " fma.rn.f32x2 d, a, b, c;\n mov.b64 {%0, %1}, d;\n}\n"
+      : "=f"(x0), "=f"(x1)
+      : "r"(s0), "r"(s1), "f"(sl2), "f"(nlse));
+  const float p0 = ex2(x0), p1 = ex2(x1);
+  float d0, d1;
+  asm("{\n .reg .b64 a, b, c, d;\n"
+      " mov.b64 a, {%2, %3};\n mov.b64 b, {%4, %4};\n add.rn.f32x2 c, a, b;\n"
+      " mov.b64 d, {%5, %6};\n mul.rn.f32x2 c, c, d;\n mov.b64 {%0, %1}, c;\n}\n"
+      : "=f"(d0), "=f"(d1)
+      : "r"(dp0), "r"(dp1), "f"(nD), "f"(p0), "f"(p1));
+  return pack_bf16(d0, d1);
+}
+
+template <bool SPLIT>
+__global__ void __launch_bounds__(BW_NTHREADS, 1)
+    attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qlo,
+                          const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_k0,
+                          const __grid_constant__ CUtensorMap tm_v0, const __grid_constant__ CUtensorMap tm_k1,
+                          const __grid_constant__ CUtensorMap tm_v1, const __grid_constant__ CUtensorMap tm_klo,
+                          const BwdTc t) {
+  using L = DqLay<SPLIT>;
+  const BwdArgs& a = t.b;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - raw);
+  const DqBars bars{sbase + L::BAR, L::NST};
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sgen + L::TMEM_SLOT);
+  const int warp = threadIdx.x >> 5;
+  const int h = blockIdx.y;
+  const int row0 = blockIdx.x * TBM;
+  const int ntile = t.tiles_total;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bars.q_full(), 1);
+    for (int s = 0; s < L::NST; ++s) {
+      mbar_init(bars.full(s), 1);
+      mbar_init(bars.empty(s), 1);
+    }
+    mbar_init(bars.s_full(), 1);
+    mbar_init(bars.s_free(), TBM / 32);
+    mbar_init(bars.ds_full(), TBM / 32);
+    mbar_init(bars.dq_done(), 1);
+    mbar_init(bars.fin(), 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc<TMEM_COLS>(smem_u32(tmem_slot));
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (ntile > 0) {
+      const bool leader = elect_one();
+      const int qy = h * a.n_q + row0;
+      if (leader) {
+        mbar_expect_tx(bars.q_full(), L::QT * TILE);
+        tma_load_2d(sbase, &tm_q, 0, qy, bars.q_full());
+        if constexpr (SPLIT) tma_load_2d(sbase + TILE, &tm_qlo, 0, qy, bars.q_full());
+        tma_load_2d(sbase + (L::QT - 1) * TILE, &tm_do, 0, qy, bars.q_full());
+      }
+      __syncwarp();
+      int issued = 0;
+      for (int it = 0; it < ntile; ++it) {
+        const int s = it % L::NST;
+        if (it >= L::NST &&
+            !__all_sync(0xffffffffu, mbar_wait(bars.empty(s), ((it / L::NST) - 1) & 1, t.err)))
+          break;
+        long long kb;
+        const int seg = bw_seg(t, it, kb);
+        const int y = static_cast<int>(static_cast<long long>(h) * a.n_k[seg] + kb);
+        const uint32_t st = sbase + L::KV + s * L::STAGE;
+        if (leader) {
+          mbar_expect_tx(bars.full(s), L::KT * TILE);
+          tma_load_2d(st, seg ? &tm_k1 : &tm_k0, 0, y, bars.full(s));
+          if constexpr (SPLIT) tma_load_2d(st + TILE, &tm_klo, 0, y, bars.full(s));
+          tma_load_2d(st + (L::KT - 1) * TILE, seg ? &tm_v1 : &tm_v0, 0, y, bars.full(s));
+        }
+        __syncwarp();
+        ++issued;
+      }
+      for (int it = max(0, issued - L::NST); it < issued; ++it)
+        mbar_wait(bars.full(it % L::NST), (it / L::NST) & 1, t.err);
+      mbar_wait(bars.q_full(), 0, t.err);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (ntile > 0) {
+      const bool leader = elect_one();
+      constexpr uint32_t T16 = TILE >> 4, ST16 = L::STAGE >> 4;
+      const uint64_t dq0 = sdesc_sw128(sbase, 16, 1024);                           // Q hi
+      const uint64_t ddo = dq0 + (L::QT - 1) * T16;                               // dO
+      const uint64_t dk0 = sdesc_sw128(sbase + L::KV, 16, 1024);                  // K hi, K-major
+      const uint64_t dv0 = dk0 + (L::KT - 1) * T16;                               // V, K-major
+      const uint64_t dkb0 = sdesc_sw128(sbase + L::KV, 8192, 1024);               // K hi, MN-major
+      bool ok = __all_sync(0xffffffffu, mbar_wait(bars.q_full(), 0, t.err));
+      tc_fence_after();
+      for (int j = 0; ok && j <= ntile; ++j) {
+        if (j < ntile) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bars.full(j % L::NST), (j / L::NST) & 1, t.err));
+          if (!ok) break;
+          if (j > 0) ok = __all_sync(0xffffffffu, mbar_wait(bars.s_free(), (j - 1) & 1, t.err));
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t dk = dk0 + (j % L::NST) * ST16, dv = dv0 + (j % L::NST) * ST16;
+          if (leader) {
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              mma_bf16_ss(tmem, dq0 + 2 * ks, dk + 2 * ks, IDESC_QK, ks > 0 ? 1u : 0u);
+              if constexpr (SPLIT) {
+                mma_bf16_ss(tmem, dq0 + 2 * ks, dk + T16 + 2 * ks, IDESC_QK, 1u);
+                mma_bf16_ss(tmem, dq0 + T16 + 2 * ks, dk + 2 * ks, IDESC_QK, 1u);
+              }
+            }
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) mma_bf16_ss(tmem + 128, ddo + 2 * ks, dv + 2 * ks, IDESC_QK, ks > 0 ? 1u : 0u);
+            mma_commit(bars.s_full());
+          }
+          __syncwarp();
+        }
+        if (j > 0) {
+          // dQ += dS_{j-1} K_{j-1}: dS read from TMEM (TS form), K MN-major
+          ok = __all_sync(0xffffffffu, mbar_wait(bars.ds_full(), (j - 1) & 1, t.err));
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t dkb = dkb0 + ((j - 1) % L::NST) * ST16;
+          if (leader) {
+#pragma unroll
+            for (int ks = 0; ks < TBN / 16; ++ks)
+              mma_bf16_ts(tmem + 256, tmem + 320 + 8 * ks, dkb + ks * 128, IDESC_PV, (j > 1 || ks > 0) ? 1u : 0u);
+            mma_commit(bars.dq_done());
+            mma_commit(bars.empty((j - 1) % L::NST));
+          }
+          __syncwarp();
+        }
+      }
+      if (leader) mma_commit(bars.fin());
+      __syncwarp();
+      mbar_wait(bars.fin(), 0, t.err);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int r = threadIdx.x;                        // row in the tile = TMEM lane
+    const int row = row0 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tS = tmem + lane_off, tP = tS + 128, tQ = tS + 256, tD = tS + 320;
+    const float sl2 = a.scale_log2;
+    const bool rv = row < a.n_q;
+    // rows past the end: lse = +inf makes P (and dS) zero
+    const float nlse = rv ? -a.lse2[static_cast<long long>(h) * a.n_q + row] : -INFINITY;
+    const float nD = rv ? -a.Dv[static_cast<long long>(h) * a.n_q + row] : 0.f;
+    bool ok = true;
+    for (int j = 0; j < ntile; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bars.s_full(), j & 1, t.err));
+      if (!ok) break;
+      tc_fence_after();
+      long long kb;
+      const int seg = bw_seg(t, j, kb);
+      const int nk = a.n_k[seg];
+      const int km = a.kmask[seg];
+      uint32_t vm[4] = {~0u, ~0u, ~0u, ~0u};
+      if (km != MASK_NONE || kb + TBN > nk) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) vm[c] = chunk_valid(km, a.g, nk, kb + 32 * c);
+      }
+#pragma unroll 1
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t sv[64], pv[64];
+        tmem_ld64(tS + 64 * hf, sv);
+        tmem_ld64(tP + 64 * hf, pv);
+        tmem_wait_ld();
+        if (hf == 1) {
+          tc_fence_before();
+          warp_arrive(bars.s_free());
+        }
+        const uint32_t m0 = sel_if(hf, vm[2], vm[0]), m1 = sel_if(hf, vm[3], vm[1]);
+        if (m0 != ~0u) apply_mask(sv, m0);
+        if (m1 != ~0u) apply_mask(sv + 32, m1);
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 64; e += 2) pk[e >> 1] = ds_pair(sv[e], sv[e + 1], pv[e], pv[e + 1], sl2, nlse, nD);
+        // dS_i is free once dQ of the previous tile has completed
+        if (hf == 0 && j > 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bars.dq_done(), (j - 1) & 1, t.err));
+          if (!ok) break;
+        }
+        tmem_st32(tD + 32 * hf, pk);
+      }
+      if (!ok) break;
+      tmem_wait_st();
+      tc_fence_before();
+      warp_arrive(bars.ds_full());
+    }
+    if (ok && ntile > 0) ok = mbar_wait(bars.dq_done(), (ntile - 1) & 1, t.err);
+    ok = __all_sync(0xffffffffu, ok);
+    tc_fence_after();
+    if (ok && ntile > 0) {
+      float* out = a.dq + h * a.dq_hs + static_cast<long long>(rv ? row : 0) * D;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t w[32];
+        tmem_ld32(tQ + 32 * c, w);            // warp-collective: every lane loads
+        tmem_wait_ld();
+        if (rv) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            float4 v = make_float4(__uint_as_float(w[e]) * a.scale, __uint_as_float(w[e + 1]) * a.scale,
+                                   __uint_as_float(w[e + 2]) * a.scale, __uint_as_float(w[e + 3]) * a.scale);
+            float4* p = reinterpret_cast<float4*>(out + 32 * c + e);
+            if (a.dq_accum) {
+              const float4 o = *p;
+              v.x += o.x; v.y += o.y; v.z += o.z; v.w += o.w;
+            }
+            *p = v;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc<TMEM_COLS>(tmem);
+}
+
+template <bool SPLIT>
+cudaError_t launch_dq_tc(const BwdTc& t, const CUtensorMap* maps, cudaStream_t st) {
+  const int sm = DqLay<SPLIT>::BYTES;
+  cudaError_t e = cudaFuncSetAttribute(attn_bwd_dq_tc_kernel<SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+  if (e != cudaSuccess) return e;
+  dim3 grid((t.b.n_q + TBM - 1) / TBM, t.b.H);
+  attn_bwd_dq_tc_kernel<SPLIT><<<grid, BW_NTHREADS, sm, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5],
+                                                              maps[6], maps[7], t);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 int attn_tc_tiles(long long n) { return static_cast<int>((n + TBN - 1) / TBN); }
@@ -772,6 +1067,35 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
   if (a.kc <= 32) return launch_kc2<32>(a, maps, st);
   if (a.kc <= 64) return launch_kc2<64>(a, maps, st);
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_attn_bwd_dq_tc(const BwdArgs& b, int* err, cudaStream_t st) {
+  const long long H = b.H;
+  // the tensor maps address rows as head * rows + row: heads must be packed
+  if (b.q_hs != static_cast<long long>(b.n_q) * D || b.do_hs != b.q_hs) return cudaErrorInvalidValue;
+  for (int s = 0; s < b.nseg; ++s)
+    if (b.kv_hs[s] != static_cast<long long>(b.n_k[s]) * D) return cudaErrorInvalidValue;
+  const bool split = b.q_lo != nullptr;
+  if (split && (b.k_lo == nullptr || b.nseg != 1)) return cudaErrorInvalidValue;
+  CUtensorMap maps[8];
+  memset(maps, 0, sizeof(maps));
+  if (!make_map(&maps[0], b.q, H * b.n_q) || !make_map(&maps[2], b.dO, H * b.n_q)) return cudaErrorInvalidValue;
+  maps[1] = maps[0];
+  if (split && !make_map(&maps[1], b.q_lo, H * b.n_q)) return cudaErrorInvalidValue;
+  if (!make_map(&maps[3], b.k[0], H * b.n_k[0]) || !make_map(&maps[4], b.v[0], H * b.n_k[0]))
+    return cudaErrorInvalidValue;
+  maps[5] = maps[3];
+  maps[6] = maps[4];
+  if (b.nseg > 1 && (!make_map(&maps[5], b.k[1], H * b.n_k[1]) || !make_map(&maps[6], b.v[1], H * b.n_k[1])))
+    return cudaErrorInvalidValue;
+  maps[7] = maps[3];
+  if (split && !make_map(&maps[7], b.k_lo, H * b.n_k[0])) return cudaErrorInvalidValue;
+  BwdTc t;
+  t.b = b;
+  t.tiles0 = attn_tc_tiles(b.n_k[0]);
+  t.tiles_total = t.tiles0 + (b.nseg > 1 ? attn_tc_tiles(b.n_k[1]) : 0);
+  t.err = err;
+  return split ? launch_dq_tc<true>(t, maps, st) : launch_dq_tc<false>(t, maps, st);
 }
 
 }  // namespace gsa

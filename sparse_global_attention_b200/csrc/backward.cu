@@ -316,6 +316,17 @@ __global__ void __launch_bounds__(128) attn_bwd_dkv_kernel(const BwdArgs a, int 
 constexpr int DQ_SMEM = 3 * TB + 2 * 3 * TB + 2 * BT;
 constexpr int DKV_SMEM = 3 * TB + 2 * 3 * TB + 2 * 2 * BT * 4;
 
+cudaError_t launch_attn_bwd_dkv(const BwdArgs& a, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DKV_SMEM);
+  if (e != cudaSuccess) return e;
+  for (int seg = 0; seg < a.nseg; ++seg) {
+    if (!a.dk[seg]) continue;
+    attn_bwd_dkv_kernel<<<dim3(static_cast<unsigned>((a.n_k[seg] + BT - 1) / BT), a.H), 128, DKV_SMEM, st>>>(a, seg);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 cudaError_t launch_attn_bwd(const BwdArgs& a, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(attn_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DQ_SMEM);
   if (e != cudaSuccess) return e;
