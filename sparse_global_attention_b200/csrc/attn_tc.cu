@@ -1012,6 +1012,287 @@ cudaError_t launch_dq_tc(const BwdTc& t, const CUtensorMap* maps, cudaStream_t s
   return cudaGetLastError();
 }
 
+// ==== attention backward on tcgen05: dK, dV ==================================
+// Per CTA one 128-key tile of one key segment (thread = key = TMEM lane)
+// against every query tile: S^T = K Q^T (split guide where the forward had
+// one) and dP^T = V dO^T into TMEM; the softmax warps form
+// P^T = exp2(S^T * scale * log2 e - lse2[query]) and dS^T = P^T o (dP^T - D[query])
+// in bf16 pairs; dV += P^T dO and dK += dS^T Q run in the TS form with dO and Q
+// as MN-major operands.  lse2 and D of a query tile sit in shared memory next
+// to its tiles (written by the producer warp).
+// TMEM: S^T [0,128), dP^T [128,256), dV [256,320), dK [320,384),
+// P^T [384,448), dS^T [448,512).
+template <bool SPLIT>
+struct DkvLay {
+  static constexpr int NST = 3;
+  static constexpr int KT = SPLIT ? 3 : 2;     // resident: K hi, [K lo], V
+  static constexpr int QT = SPLIT ? 3 : 2;     // per stage: Q hi, [Q lo], dO
+  static constexpr int KV = KT * TILE;
+  static constexpr int LD = QT * TILE;         // -lse2[128] then -D[128] after the stage's tiles
+  static constexpr int STAGE = QT * TILE + 1024;
+  static constexpr int BAR = KV + NST * STAGE;
+  // k_full, full[NST], empty[NST], s_full, s_free, pds_full, kv_done, fin
+  static constexpr int NBAR = 1 + 2 * NST + 5;
+  static constexpr int TMEM_SLOT = BAR + NBAR * 8;
+  static constexpr int BYTES = TMEM_SLOT + 16 + 1024;
+};
+
+template <bool SPLIT>
+__global__ void __launch_bounds__(BW_NTHREADS, 1)
+    attn_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qlo,
+                           const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_k,
+                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_klo,
+                           const BwdTc t, const int seg) {
+  using L = DkvLay<SPLIT>;
+  const BwdArgs& a = t.b;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - raw);
+  const DqBars bars{sbase + L::BAR, L::NST};      // q_full() is the resident K/V tiles here
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sgen + L::TMEM_SLOT);
+  const int warp = threadIdx.x >> 5;
+  const int h = blockIdx.y;
+  const int key0 = blockIdx.x * TBM;
+  const int nk = a.n_k[seg];
+  const int ntile = (a.n_q + TBN - 1) / TBN;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bars.q_full(), 1);
+    for (int s = 0; s < L::NST; ++s) {
+      mbar_init(bars.full(s), 1);
+      mbar_init(bars.empty(s), 1);
+    }
+    mbar_init(bars.s_full(), 1);
+    mbar_init(bars.s_free(), TBM / 32);
+    mbar_init(bars.ds_full(), TBM / 32);
+    mbar_init(bars.dq_done(), 1);
+    mbar_init(bars.fin(), 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc<TMEM_COLS>(smem_u32(tmem_slot));
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (ntile > 0) {
+      const int lane = threadIdx.x & 31;
+      const bool leader = elect_one();
+      const int ky = h * nk + key0;
+      if (leader) {
+        mbar_expect_tx(bars.q_full(), L::KT * TILE);
+        tma_load_2d(sbase, &tm_k, 0, ky, bars.q_full());
+        if constexpr (SPLIT) tma_load_2d(sbase + TILE, &tm_klo, 0, ky, bars.q_full());
+        tma_load_2d(sbase + (L::KT - 1) * TILE, &tm_v, 0, ky, bars.q_full());
+      }
+      __syncwarp();
+      int issued = 0;
+      for (int it = 0; it < ntile; ++it) {
+        const int s = it % L::NST;
+        if (it >= L::NST &&
+            !__all_sync(0xffffffffu, mbar_wait(bars.empty(s), ((it / L::NST) - 1) & 1, t.err)))
+          break;
+        const uint32_t st = sbase + L::KV + s * L::STAGE;
+        // -lse2 and -D of the tile's queries (rows past the end: P = 0)
+        float* ld = reinterpret_cast<float*>(sgen + L::KV + s * L::STAGE + L::LD);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int row = it * TBN + 32 * q + lane;
+          const bool ok = row < a.n_q;
+          const long long gi = static_cast<long long>(h) * a.n_q + (ok ? row : 0);
+          ld[32 * q + lane] = ok ? -a.lse2[gi] : -INFINITY;
+          ld[TBN + 32 * q + lane] = ok ? -a.Dv[gi] : 0.f;
+        }
+        __syncwarp();
+        const int y = h * a.n_q + it * TBN;
+        if (leader) {
+          mbar_expect_tx(bars.full(s), L::QT * TILE);
+          tma_load_2d(st, &tm_q, 0, y, bars.full(s));
+          if constexpr (SPLIT) tma_load_2d(st + TILE, &tm_qlo, 0, y, bars.full(s));
+          tma_load_2d(st + (L::QT - 1) * TILE, &tm_do, 0, y, bars.full(s));
+        }
+        __syncwarp();
+        ++issued;
+      }
+      for (int it = max(0, issued - L::NST); it < issued; ++it)
+        mbar_wait(bars.full(it % L::NST), (it / L::NST) & 1, t.err);
+      mbar_wait(bars.q_full(), 0, t.err);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (ntile > 0) {
+      const bool leader = elect_one();
+      constexpr uint32_t T16 = TILE >> 4, ST16 = L::STAGE >> 4;
+      const uint64_t dk = sdesc_sw128(sbase, 16, 1024);                           // K hi (A)
+      const uint64_t dvv = dk + (L::KT - 1) * T16;                                // V (A)
+      const uint64_t dq0 = sdesc_sw128(sbase + L::KV, 16, 1024);                  // Q hi, K-major (B)
+      const uint64_t ddo0 = dq0 + (L::QT - 1) * T16;                              // dO, K-major (B)
+      const uint64_t dqm0 = sdesc_sw128(sbase + L::KV, 8192, 1024);               // Q hi, MN-major (B)
+      const uint64_t ddom0 = dqm0 + (L::QT - 1) * T16;                            // dO, MN-major (B)
+      bool ok = __all_sync(0xffffffffu, mbar_wait(bars.q_full(), 0, t.err));
+      tc_fence_after();
+      for (int j = 0; ok && j <= ntile; ++j) {
+        if (j < ntile) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bars.full(j % L::NST), (j / L::NST) & 1, t.err));
+          if (!ok) break;
+          if (j > 0) ok = __all_sync(0xffffffffu, mbar_wait(bars.s_free(), (j - 1) & 1, t.err));
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t dq = dq0 + (j % L::NST) * ST16, ddo = ddo0 + (j % L::NST) * ST16;
+          if (leader) {
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              mma_bf16_ss(tmem, dk + 2 * ks, dq + 2 * ks, IDESC_QK, ks > 0 ? 1u : 0u);
+              if constexpr (SPLIT) {
+                mma_bf16_ss(tmem, dk + T16 + 2 * ks, dq + 2 * ks, IDESC_QK, 1u);
+                mma_bf16_ss(tmem, dk + 2 * ks, dq + T16 + 2 * ks, IDESC_QK, 1u);
+              }
+            }
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) mma_bf16_ss(tmem + 128, dvv + 2 * ks, ddo + 2 * ks, IDESC_QK, ks > 0 ? 1u : 0u);
+            mma_commit(bars.s_full());
+          }
+          __syncwarp();
+        }
+        if (j > 0) {
+          // dV += P^T dO, dK += dS^T Q of tile j-1 (TS form, dO and Q MN-major)
+          ok = __all_sync(0xffffffffu, mbar_wait(bars.ds_full(), (j - 1) & 1, t.err));
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t dqm = dqm0 + ((j - 1) % L::NST) * ST16, ddom = ddom0 + ((j - 1) % L::NST) * ST16;
+          if (leader) {
+#pragma unroll
+            for (int ks = 0; ks < TBN / 16; ++ks) {
+              mma_bf16_ts(tmem + 256, tmem + 384 + 8 * ks, ddom + ks * 128, IDESC_PV, (j > 1 || ks > 0) ? 1u : 0u);
+              mma_bf16_ts(tmem + 320, tmem + 448 + 8 * ks, dqm + ks * 128, IDESC_PV, (j > 1 || ks > 0) ? 1u : 0u);
+            }
+            mma_commit(bars.dq_done());
+            mma_commit(bars.empty((j - 1) % L::NST));
+          }
+          __syncwarp();
+        }
+      }
+      if (leader) mma_commit(bars.fin());
+      __syncwarp();
+      mbar_wait(bars.fin(), 0, t.err);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int r = threadIdx.x;                        // key in the tile = TMEM lane
+    const int key = key0 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tS = tmem + lane_off, tP = tS + 128, tV = tS + 256, tK = tS + 320, tPT = tS + 384,
+                   tDS = tS + 448;
+    const float sl2 = a.scale_log2;
+    const bool kv = key < nk && key_valid(a.kmask[seg], a.g, key);
+    bool ok = true;
+    for (int j = 0; j < ntile; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bars.s_full(), j & 1, t.err));
+      if (!ok) break;
+      // the producer's lse2/D stores of this stage: acquired through its full barrier
+      // (complete by now; the stage cannot be refilled before this tile's dK/dV MMAs)
+      ok = __all_sync(0xffffffffu, mbar_wait(bars.full(j % L::NST), (j / L::NST) & 1, t.err));
+      if (!ok) break;
+      tc_fence_after();
+      const float* ld = reinterpret_cast<const float*>(sgen + L::KV + (j % L::NST) * L::STAGE + L::LD);
+#pragma unroll 1
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t sv[64], pv[64];
+        tmem_ld64(tS + 64 * hf, sv);
+        tmem_ld64(tP + 64 * hf, pv);
+        tmem_wait_ld();
+        if (hf == 1) {
+          tc_fence_before();
+          warp_arrive(bars.s_free());
+        }
+        if (!kv) apply_mask(sv, 0u), apply_mask(sv + 32, 0u);
+        uint32_t pk[32], dk[32];
+#pragma unroll
+        for (int e = 0; e < 64; e += 2) {
+          const float2 nl = *reinterpret_cast<const float2*>(ld + 64 * hf + e);
+          const float2 nd = *reinterpret_cast<const float2*>(ld + TBN + 64 * hf + e);
+          float x0, x1;
+          asm("{\n .reg .b64 a, b, c, d;\n"
+              " mov.b64 a, {%2, %3};\n mov.b64 b, {%4, %4};\n mov.b64 c, {%5, %6};\n"
+              " fma.rn.f32x2 d, a, b, c;\n mov.b64 {%0, %1}, d;\n}\n"
+              : "=f"(x0), "=f"(x1)
+              : "r"(sv[e]), "r"(sv[e + 1]), "f"(sl2), "f"(nl.x), "f"(nl.y));
+          const float p0 = ex2(x0), p1 = ex2(x1);
+          float d0, d1;
+          asm("{\n .reg .b64 a, b, c, d;\n"
+              " mov.b64 a, {%2, %3};\n mov.b64 b, {%4, %5};\n add.rn.f32x2 c, a, b;\n"
+              " mov.b64 d, {%6, %7};\n mul.rn.f32x2 c, c, d;\n mov.b64 {%0, %1}, c;\n}\n"
+              : "=f"(d0), "=f"(d1)
+              : "r"(pv[e]), "r"(pv[e + 1]), "f"(nd.x), "f"(nd.y), "f"(p0), "f"(p1));
+          pk[e >> 1] = pack_bf16(p0, p1);
+          dk[e >> 1] = pack_bf16(d0, d1);
+        }
+        // P^T and dS^T are free once dV and dK of the previous tile have completed
+        if (hf == 0 && j > 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bars.dq_done(), (j - 1) & 1, t.err));
+          if (!ok) break;
+        }
+        tmem_st32(tPT + 32 * hf, pk);
+        tmem_st32(tDS + 32 * hf, dk);
+      }
+      if (!ok) break;
+      tmem_wait_st();
+      tc_fence_before();
+      warp_arrive(bars.ds_full());
+    }
+    if (ok && ntile > 0) ok = mbar_wait(bars.dq_done(), (ntile - 1) & 1, t.err);
+    ok = __all_sync(0xffffffffu, ok);
+    tc_fence_after();
+    if (ok && ntile > 0) {
+      const bool wr = key < nk;
+      const long long off = h * a.dkv_hs[seg] + static_cast<long long>(wr ? key : 0) * D;
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {
+        float* out = (which ? a.dk[seg] : a.dv[seg]) + off;
+        const float sc = which ? a.scale : 1.f;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t w[32];
+          tmem_ld32((which ? tK : tV) + 32 * c, w);       // warp-collective: every lane loads
+          tmem_wait_ld();
+          if (wr) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              float4 v = make_float4(__uint_as_float(w[e]) * sc, __uint_as_float(w[e + 1]) * sc,
+                                     __uint_as_float(w[e + 2]) * sc, __uint_as_float(w[e + 3]) * sc);
+              float4* p = reinterpret_cast<float4*>(out + 32 * c + e);
+              if (a.dkv_accum) {
+                const float4 o = *p;
+                v.x += o.x; v.y += o.y; v.z += o.z; v.w += o.w;
+              }
+              *p = v;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc<TMEM_COLS>(tmem);
+}
+
+template <bool SPLIT>
+cudaError_t launch_dkv_tc(const BwdTc& t, const CUtensorMap* maps, int seg, cudaStream_t st) {
+  const int sm = DkvLay<SPLIT>::BYTES;
+  cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkv_tc_kernel<SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+  if (e != cudaSuccess) return e;
+  dim3 grid((t.b.n_k[seg] + TBM - 1) / TBM, t.b.H);
+  attn_bwd_dkv_tc_kernel<SPLIT><<<grid, BW_NTHREADS, sm, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5],
+                                                               t, seg);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 int attn_tc_tiles(long long n) { return static_cast<int>((n + TBN - 1) / TBN); }
@@ -1096,6 +1377,35 @@ cudaError_t launch_attn_bwd_dq_tc(const BwdArgs& b, int* err, cudaStream_t st) {
   t.tiles_total = t.tiles0 + (b.nseg > 1 ? attn_tc_tiles(b.n_k[1]) : 0);
   t.err = err;
   return split ? launch_dq_tc<true>(t, maps, st) : launch_dq_tc<false>(t, maps, st);
+}
+
+cudaError_t launch_attn_bwd_dkv_tc(const BwdArgs& b, int* err, cudaStream_t st) {
+  const long long H = b.H;
+  if (b.q_hs != static_cast<long long>(b.n_q) * D || b.do_hs != b.q_hs) return cudaErrorInvalidValue;
+  for (int s = 0; s < b.nseg; ++s)
+    if (b.kv_hs[s] != static_cast<long long>(b.n_k[s]) * D) return cudaErrorInvalidValue;
+  const bool split = b.q_lo != nullptr;
+  if (split && (b.k_lo == nullptr || b.nseg != 1)) return cudaErrorInvalidValue;
+  CUtensorMap maps[6];
+  memset(maps, 0, sizeof(maps));
+  if (!make_map(&maps[0], b.q, H * b.n_q) || !make_map(&maps[2], b.dO, H * b.n_q)) return cudaErrorInvalidValue;
+  maps[1] = maps[0];
+  if (split && !make_map(&maps[1], b.q_lo, H * b.n_q)) return cudaErrorInvalidValue;
+  BwdTc t;
+  t.b = b;
+  t.tiles0 = 0;
+  t.tiles_total = 0;
+  t.err = err;
+  for (int seg = 0; seg < b.nseg; ++seg) {
+    if (!b.dk[seg]) continue;
+    if (!make_map(&maps[3], b.k[seg], H * b.n_k[seg]) || !make_map(&maps[4], b.v[seg], H * b.n_k[seg]))
+      return cudaErrorInvalidValue;
+    maps[5] = maps[3];
+    if (split && !make_map(&maps[5], b.k_lo, H * b.n_k[0])) return cudaErrorInvalidValue;
+    const cudaError_t e = split ? launch_dkv_tc<true>(t, maps, seg, st) : launch_dkv_tc<false>(t, maps, seg, st);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace gsa

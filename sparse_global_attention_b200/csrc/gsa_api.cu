@@ -734,7 +734,7 @@ int gsa_backward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void*
   ba.dq = dqc; ba.dq_hs = rhs; ba.dq_accum = 0;
   ba.dk[0] = dkc; ba.dv[0] = dvc; ba.dkv_hs[0] = rhs; ba.dkv_accum = 0;
   ba.H = H; ba.g = g; ba.scale_log2 = scale * LOG2E; ba.scale = scale;
-  if (launch_attn_bwd_dq_tc(ba, err, st) != cudaSuccess || launch_attn_bwd_dkv(ba, st) != cudaSuccess)
+  if (launch_attn_bwd_dq_tc(ba, err, st) != cudaSuccess || launch_attn_bwd_dkv_tc(ba, err, st) != cudaSuccess)
     return GSA_ERR_CUDA;
   prof.mark("bwd_comp_attn");
 
@@ -768,7 +768,7 @@ int gsa_backward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void*
     bs.dk[0] = dk_spec; bs.dv[0] = dv_spec; bs.dkv_hs[0] = shs;
     bs.dk[1] = dk_img; bs.dv[1] = dv_img; bs.dkv_hs[1] = ihs; bs.dkv_accum = 1;
     bs.H = H; bs.g = g; bs.scale_log2 = scale * LOG2E; bs.scale = scale;
-    if (launch_attn_bwd_dq_tc(bs, err, st) != cudaSuccess || launch_attn_bwd_dkv(bs, st) != cudaSuccess)
+    if (launch_attn_bwd_dq_tc(bs, err, st) != cudaSuccess || launch_attn_bwd_dkv_tc(bs, err, st) != cudaSuccess)
       return GSA_ERR_CUDA;
     prof.mark("bwd_special");
   }

@@ -170,6 +170,8 @@ cudaError_t launch_attn_bwd_dkv(const BwdArgs& a, cudaStream_t st);
 // dQ on tcgen05/TMEM/TMA: 128 query rows per CTA; heads packed (q_hs = n_q * 64,
 // kv_hs = n_k * 64); split scores (q_lo, k_lo) with one key segment only
 cudaError_t launch_attn_bwd_dq_tc(const BwdArgs& a, int* err, cudaStream_t st);
+// dK/dV on tcgen05: 128 keys per CTA, one launch per key segment (same layout rules)
+cudaError_t launch_attn_bwd_dkv_tc(const BwdArgs& a, int* err, cudaStream_t st);
 
 // selection + gate backward: one warp per window (s <= 4)
 struct SelBwdArgs {

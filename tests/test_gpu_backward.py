@@ -20,7 +20,10 @@ SMALL = GSAConfig("bwd_small", 3, 12, 12, 12, 12, 2, 2, 64, 4, 4, "bf16")
 MULTI = GSAConfig("bwd_multi_tile", 6, 24, 24, 24, 24, 3, 2, 64, 4, 16, "bf16")
 S2 = GSAConfig("bwd_s2", 2, 10, 14, 10, 14, 1, 2, 64, 2, 12, "bf16")
 VGGT = GSAConfig("bwd_pad_vggt", 5, 10, 11, 12, 12, 3, 2, 64, 4, 6, "bf16", (0, 3))
-CASES = [SMALL, MULTI, S2, VGGT]
+# 600 regions and 528 special rows: five 128-row tiles each, so the three-stage
+# TMA rings of the tcgen05 dQ and dK/dV kernels wrap around
+WRAP = GSAConfig("bwd_ring_wrap", 24, 20, 20, 20, 20, 22, 2, 64, 4, 8, "bf16")
+CASES = [SMALL, MULTI, S2, VGGT, WRAP]
 
 
 def _close(name, got, want):
