@@ -92,10 +92,14 @@ def algorithmic_work(cfg, kc):
     return w
 
 
+# the sources the tcgen05 attention kernels (K2, K5) are compiled from
+KERNEL_SOURCES = ("attn_tc.cu", "tc_ptx.cuh", "gsa_common.cuh", "gsa_kernels.h")
+
+
 def kernel_source_sha():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sparse_global_attention_b200", "csrc")
-    for n in sorted(os.listdir(csrc)):
+    for n in KERNEL_SOURCES:
         with open(os.path.join(csrc, n), "rb") as f:
             h.update(n.encode())
             h.update(f.read())
