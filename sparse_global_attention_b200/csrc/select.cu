@@ -472,6 +472,12 @@ __device__ __forceinline__ void ldsm_pitch32(uint32_t base, int r0, uint32_t (&a
   ldsm_x4(addr, a[0], a[1], a[2], a[3]);
 }
 
+// four consecutive floats added to global memory in one vector reduction (16-byte aligned)
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
 template <int S>
 __global__ void __launch_bounds__(SEL_WARPS * 32) sel_bwd_kernel(const SelBwdArgs b) {
   const SelArgs& a = b.s;
@@ -843,19 +849,25 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) sel_bwd_kernel(const SelBwdArg
         mma_bf16(acc[2 * dp2 + 1], af, b2, b3);
       }
       const float mul = isv ? 1.f : scale;
-#pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-        const int key = 16 * mt + g + 8 * rr;
-        if (!sValid[st * SEL_BN + key]) continue;
+      // lanes t and t^1 hold two columns each of the same four: one shuffle gives the
+      // even lane four columns of row g and the odd lane four of row g + 8, so each
+      // lane adds one 16-byte vector per n-tile (half the reductions of float2 atomics)
+      const int rr = t & 1;
+      const int key = 16 * mt + g + 8 * rr;
+      float* base = nullptr;
+      if (sValid[st * SEL_BN + key]) {
         long long off;
         bool spec;
         key_src<S>(a, sReg, blk * SEL_BN + key, nk_dyn, nkeys, off, spec);
-        float* base = spec ? (isv ? dvsh : dksh) : (isv ? dvh : dkh);
-        if (!base) continue;
-        base += off * D + 2 * t;
+        base = spec ? (isv ? dvsh : dksh) : (isv ? dvh : dkh);
+        if (base) base += off * D + 4 * (t >> 1);
+      }
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-          atomicAdd(reinterpret_cast<float2*>(base + 8 * nt), make_float2(acc[nt][2 * rr] * mul, acc[nt][2 * rr + 1] * mul));
+      for (int nt = 0; nt < 8; ++nt) {
+        const float x0 = acc[nt][0] * mul, x1 = acc[nt][1] * mul, y0 = acc[nt][2] * mul, y1 = acc[nt][3] * mul;
+        const float o0 = __shfl_xor_sync(0xffffffffu, rr ? x0 : y0, 1);
+        const float o1 = __shfl_xor_sync(0xffffffffu, rr ? x1 : y1, 1);
+        if (base) red_add_v4(base + 8 * nt, rr ? o0 : x0, rr ? o1 : x1, rr ? y0 : o0, rr ? y1 : o1);
       }
     }
   }
