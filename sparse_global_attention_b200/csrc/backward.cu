@@ -11,11 +11,8 @@
 //              D = rowsum(dO o O),  dS = P o (dO V^T - D),
 //              dQ = scale dS K,  dK = scale dS^T Q,  dV = P^T dO
 //   pool       each valid token of region r gets dX_comp[r] / |valid tokens of r|
-// Kernels:
-//   attn_bwd_dq / attn_bwd_dkv  dense attention backward (compressed branch,
-//       special tokens), flash style: P is recomputed tile by tile from the
-//       forward's log-sum-exp; dQ by query tiles, dK/dV by key tiles, so no
-//       gradient needs atomics.  m16n8k16 bf16 MMAs, fp32 accumulation.
+// Kernels (the dense attention backward of the compressed branch and the
+// special tokens runs on tcgen05, in attn_tc.cu):
 //   sel_bwd     one warp per window: recomputes the selection forward, runs the
 //       gate backward, writes dO'_comp of its region and dq of its tokens, and
 //       adds dK/dV of its keys (shared by many windows) with fp32 atomics.
@@ -24,323 +21,6 @@
 #include "gsa_kernels.h"
 
 namespace gsa {
-
-namespace {
-
-constexpr int BT = 64;                  // rows per CTA tile (4 warps x 16) and keys/queries per stage
-constexpr int TB = BT * 128;            // bytes of a 64 x 64 bf16 tile
-
-// A-operand fragments (m16 x k16, 4 k-steps over d = 64) of the 16 rows of a
-// swizzled tile starting at `base`
-__device__ __forceinline__ void load_afrag(uint32_t base, uint32_t (&f)[4][4]) {
-  const int lane = threadIdx.x & 31, mi = lane >> 3, lr = lane & 7;
-#pragma unroll
-  for (int ks = 0; ks < 4; ++ks)
-    ldsm_x4(base + swz(lr + 8 * (mi & 1), 2 * ks + (mi >> 1)), f[ks][0], f[ks][1], f[ks][2], f[ks][3]);
-}
-
-// acc[16 x 64] += A[16 x 64 (k = d)] . X^T where X is a 64-row tile [n][d]
-__device__ __forceinline__ void mma_xt(float (&acc)[8][4], const uint32_t (&a)[4][4], uint32_t xt) {
-  const int lane = threadIdx.x & 31, mi = lane >> 3, lr = lane & 7;
-#pragma unroll
-  for (int ks = 0; ks < 4; ++ks)
-#pragma unroll
-    for (int np = 0; np < 4; ++np) {
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4(xt + swz(16 * np + lr + 8 * (mi >> 1), 2 * ks + (mi & 1)), b0, b1, b2, b3);
-      mma_bf16(acc[2 * np], a[ks], b0, b1);
-      mma_bf16(acc[2 * np + 1], a[ks], b2, b3);
-    }
-}
-
-// acc[16 x 64 (d)] += A[16 x 64 (k = rows of X)] . X where X is a 64-row tile [k][d]
-__device__ __forceinline__ void mma_x(float (&acc)[8][4], const uint32_t (&a)[4][4], uint32_t x) {
-  const int lane = threadIdx.x & 31, mi = lane >> 3, lr = lane & 7;
-#pragma unroll
-  for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-    for (int dp = 0; dp < 4; ++dp) {
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4_t(x + swz(16 * kk + lr + 8 * (mi & 1), 2 * dp + (mi >> 1)), b0, b1, b2, b3);
-      mma_bf16(acc[2 * dp], a[kk], b0, b1);
-      mma_bf16(acc[2 * dp + 1], a[kk], b2, b3);
-    }
-}
-
-// C fragments of a 16 x 64 product as bf16 A fragments (k = its 64 columns)
-__device__ __forceinline__ void c_to_a(const float (&c)[8][4], uint32_t (&a)[4][4]) {
-#pragma unroll
-  for (int kk = 0; kk < 4; ++kk) {
-    a[kk][0] = pack_bf16(c[2 * kk][0], c[2 * kk][1]);
-    a[kk][1] = pack_bf16(c[2 * kk][2], c[2 * kk][3]);
-    a[kk][2] = pack_bf16(c[2 * kk + 1][0], c[2 * kk + 1][1]);
-    a[kk][3] = pack_bf16(c[2 * kk + 1][2], c[2 * kk + 1][3]);
-  }
-}
-
-__device__ __forceinline__ void zero(float (&c)[8][4]) {
-#pragma unroll
-  for (int i = 0; i < 8; ++i) c[i][0] = c[i][1] = c[i][2] = c[i][3] = 0.f;
-}
-
-// rows [row0, row0 + 64) of a [n][64] bf16 tensor into a swizzled tile; rows past n read zeros
-__device__ __forceinline__ void tile_load(uint32_t dst, const __nv_bfloat16* src, long long row0, long long n) {
-#pragma unroll
-  for (int it = 0; it < (BT * 8) / 128; ++it) {
-    const int e = threadIdx.x + it * 128;
-    const int r = e >> 3, c = e & 7;
-    const bool ok = row0 + r < n;
-    cp_async16(dst + swz(r, c), src + (ok ? row0 + r : 0) * D + c * 8, ok ? 16 : 0);
-  }
-}
-
-// segment and first key of global key tile tt
-__device__ __forceinline__ int bseg(const BwdArgs& a, int tt, long long& kb) {
-  const int t0 = static_cast<int>((a.n_k[0] + BT - 1) / BT);
-  const int seg = (a.nseg > 1 && tt >= t0) ? 1 : 0;
-  kb = static_cast<long long>(seg ? tt - t0 : tt) * BT;
-  return seg;
-}
-
-// ---- dQ: CTA = 64 query rows, loop over every key tile of both segments -------
-// smem: Q hi | Q lo | dO | 2 stages x (K hi | K lo | V) | key validity
-__global__ void __launch_bounds__(128) attn_bwd_dq_kernel(const BwdArgs a) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  const uint32_t sb = smem_u32(smem);
-  const uint32_t sQ = sb, sQl = sb + TB, sdO = sb + 2 * TB, sST = sb + 3 * TB;
-  constexpr int STG = 3 * TB;
-  uint8_t* sVal = smem + 3 * TB + 2 * STG;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int h = blockIdx.y;
-  const long long q0 = static_cast<long long>(blockIdx.x) * BT;
-  const bool split = a.q_lo != nullptr;
-
-  tile_load(sQ, a.q + h * a.q_hs, q0, a.n_q);
-  if (split) tile_load(sQl, a.q_lo + h * a.q_hs, q0, a.n_q);
-  tile_load(sdO, a.dO + h * a.do_hs, q0, a.n_q);
-  cp_async_commit();
-  const int t0 = static_cast<int>((a.n_k[0] + BT - 1) / BT);
-  const int ntile = t0 + (a.nseg > 1 ? static_cast<int>((a.n_k[1] + BT - 1) / BT) : 0);
-
-  auto issue = [&](int tt, int st) {
-    long long kb;
-    const int seg = bseg(a, tt, kb);
-    const uint32_t s = sST + st * STG;
-    tile_load(s, a.k[seg] + h * a.kv_hs[seg], kb, a.n_k[seg]);
-    if (split && seg == 0) tile_load(s + TB, a.k_lo + h * a.kv_hs[0], kb, a.n_k[0]);
-    tile_load(s + 2 * TB, a.v[seg] + h * a.kv_hs[seg], kb, a.n_k[seg]);
-    if (threadIdx.x < BT) {
-      const long long key = kb + threadIdx.x;
-      sVal[st * BT + threadIdx.x] = (key < a.n_k[seg] && key_valid(a.kmask[seg], a.g, key)) ? 1 : 0;
-    }
-  };
-  issue(0, 0);
-  cp_async_commit();
-  cp_async_wait<1>();
-  __syncthreads();
-  uint32_t qf[4][4], qlf[4][4], dof[4][4];
-  load_afrag(sQ + warp * 16 * 128, qf);
-  if (split) load_afrag(sQl + warp * 16 * 128, qlf);
-  load_afrag(sdO + warp * 16 * 128, dof);
-  float lse[2], Dr[2];
-#pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    const long long row = q0 + warp * 16 + g + 8 * rr;
-    const bool ok = row < a.n_q;
-    lse[rr] = ok ? a.lse2[h * static_cast<long long>(a.n_q) + row] : 0.f;
-    Dr[rr] = ok ? a.Dv[h * static_cast<long long>(a.n_q) + row] : 0.f;
-  }
-  float dq[8][4];
-  zero(dq);
-  for (int tt = 0; tt < ntile; ++tt) {
-    const int st = tt & 1;
-    __syncthreads();
-    if (tt + 1 < ntile) issue(tt + 1, st ^ 1);
-    cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
-    long long kb;
-    const int seg = bseg(a, tt, kb);
-    const uint32_t sK = sST + st * STG, sKl = sK + TB, sV = sK + 2 * TB;
-    float s[8][4], dp[8][4];
-    zero(s);
-    mma_xt(s, qf, sK);
-    if (split && seg == 0) {
-      mma_xt(s, qf, sKl);
-      mma_xt(s, qlf, sK);
-    }
-    zero(dp);
-    mma_xt(dp, dof, sV);
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int col = 8 * nt + 2 * t + (e & 1), rr = e >> 1;
-        const float p = sVal[st * BT + col] ? ex2(s[nt][e] * a.scale_log2 - lse[rr]) : 0.f;
-        s[nt][e] = p * (dp[nt][e] - Dr[rr]);                  // dS
-      }
-    uint32_t dsa[4][4];
-    c_to_a(s, dsa);
-    mma_x(dq, dsa, sK);
-  }
-  cp_async_wait<0>();
-#pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    const long long row = q0 + warp * 16 + g + 8 * rr;
-    if (row >= a.n_q) continue;
-    float* out = a.dq + h * a.dq_hs + row * D;
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      float2 v = make_float2(dq[nt][2 * rr] * a.scale, dq[nt][2 * rr + 1] * a.scale);
-      float2* p = reinterpret_cast<float2*>(out + 8 * nt + 2 * t);
-      if (a.dq_accum) {
-        const float2 o = *p;
-        v.x += o.x;
-        v.y += o.y;
-      }
-      *p = v;
-    }
-  }
-}
-
-// ---- dK, dV of one key segment: CTA = 64 keys, loop over every query tile -----
-// smem: K hi | K lo | V | 2 stages x (Q hi | Q lo | dO) | 2 x (lse, D) per stage
-__global__ void __launch_bounds__(128) attn_bwd_dkv_kernel(const BwdArgs a, int seg) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  const uint32_t sb = smem_u32(smem);
-  const uint32_t sK = sb, sKl = sb + TB, sV = sb + 2 * TB, sST = sb + 3 * TB;
-  constexpr int STG = 3 * TB;
-  float* sLD = reinterpret_cast<float*>(smem + 3 * TB + 2 * STG);      // [2 stages][lse 64 | D 64]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int h = blockIdx.y;
-  const long long k0 = static_cast<long long>(blockIdx.x) * BT;
-  const bool split = a.q_lo != nullptr && seg == 0;
-  const long long nk = a.n_k[seg];
-
-  tile_load(sK, a.k[seg] + h * a.kv_hs[seg], k0, nk);
-  if (split) tile_load(sKl, a.k_lo + h * a.kv_hs[0], k0, nk);
-  tile_load(sV, a.v[seg] + h * a.kv_hs[seg], k0, nk);
-  cp_async_commit();
-  const int ntile = static_cast<int>((a.n_q + BT - 1) / BT);
-  auto issue = [&](int qt, int st) {
-    const uint32_t s = sST + st * STG;
-    const long long q0 = static_cast<long long>(qt) * BT;
-    tile_load(s, a.q + h * a.q_hs, q0, a.n_q);
-    if (split) tile_load(s + TB, a.q_lo + h * a.q_hs, q0, a.n_q);
-    tile_load(s + 2 * TB, a.dO + h * a.do_hs, q0, a.n_q);
-    if (threadIdx.x < BT) {
-      const long long row = q0 + threadIdx.x;
-      const bool ok = row < a.n_q;
-      // rows past the end: lse = +inf makes P = 0
-      sLD[st * 2 * BT + threadIdx.x] = ok ? a.lse2[h * static_cast<long long>(a.n_q) + row] : INFINITY;
-      sLD[st * 2 * BT + BT + threadIdx.x] = ok ? a.Dv[h * static_cast<long long>(a.n_q) + row] : 0.f;
-    }
-  };
-  issue(0, 0);
-  cp_async_commit();
-  cp_async_wait<1>();
-  __syncthreads();
-  uint32_t kf[4][4], klf[4][4], vf[4][4];
-  load_afrag(sK + warp * 16 * 128, kf);
-  if (split) load_afrag(sKl + warp * 16 * 128, klf);
-  load_afrag(sV + warp * 16 * 128, vf);
-  bool kv[2];
-#pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    const long long key = k0 + warp * 16 + g + 8 * rr;
-    kv[rr] = key < nk && key_valid(a.kmask[seg], a.g, key);
-  }
-  float dk[8][4], dv[8][4];
-  zero(dk);
-  zero(dv);
-  for (int qt = 0; qt < ntile; ++qt) {
-    const int st = qt & 1;
-    __syncthreads();
-    if (qt + 1 < ntile) issue(qt + 1, st ^ 1);
-    cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
-    const uint32_t sQ = sST + st * STG, sQl = sQ + TB, sdO = sQ + 2 * TB;
-    const float* lse = sLD + st * 2 * BT;
-    const float* Dq = lse + BT;
-    float s[8][4], dp[8][4];
-    zero(s);
-    mma_xt(s, kf, sQ);                       // S^T = K Q^T
-    if (split) {
-      mma_xt(s, klf, sQ);
-      mma_xt(s, kf, sQl);
-    }
-    zero(dp);
-    mma_xt(dp, vf, sdO);                     // dP^T = V dO^T
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int col = 8 * nt + 2 * t + (e & 1), rr = e >> 1;
-        const float p = kv[rr] ? ex2(s[nt][e] * a.scale_log2 - lse[col]) : 0.f;
-        s[nt][e] = p;                                      // P^T
-        dp[nt][e] = p * (dp[nt][e] - Dq[col]);             // dS^T
-      }
-    uint32_t pa[4][4], dsa[4][4];
-    c_to_a(s, pa);
-    c_to_a(dp, dsa);
-    mma_x(dv, pa, sdO);                      // dV += P^T dO
-    mma_x(dk, dsa, sQ);                      // dK += dS^T Q
-  }
-  cp_async_wait<0>();
-#pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    const long long key = k0 + warp * 16 + g + 8 * rr;
-    if (key >= nk) continue;
-    float* ok_ = a.dk[seg] + h * a.dkv_hs[seg] + key * D;
-    float* ov = a.dv[seg] + h * a.dkv_hs[seg] + key * D;
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      float2 vk = make_float2(dk[nt][2 * rr] * a.scale, dk[nt][2 * rr + 1] * a.scale);
-      float2 vv = make_float2(dv[nt][2 * rr], dv[nt][2 * rr + 1]);
-      float2* pk = reinterpret_cast<float2*>(ok_ + 8 * nt + 2 * t);
-      float2* pv = reinterpret_cast<float2*>(ov + 8 * nt + 2 * t);
-      if (a.dkv_accum) {
-        const float2 ak = *pk, av = *pv;
-        vk.x += ak.x; vk.y += ak.y;
-        vv.x += av.x; vv.y += av.y;
-      }
-      *pk = vk;
-      *pv = vv;
-    }
-  }
-}
-
-}  // namespace
-
-constexpr int DQ_SMEM = 3 * TB + 2 * 3 * TB + 2 * BT;
-constexpr int DKV_SMEM = 3 * TB + 2 * 3 * TB + 2 * 2 * BT * 4;
-
-cudaError_t launch_attn_bwd_dkv(const BwdArgs& a, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DKV_SMEM);
-  if (e != cudaSuccess) return e;
-  for (int seg = 0; seg < a.nseg; ++seg) {
-    if (!a.dk[seg]) continue;
-    attn_bwd_dkv_kernel<<<dim3(static_cast<unsigned>((a.n_k[seg] + BT - 1) / BT), a.H), 128, DKV_SMEM, st>>>(a, seg);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
-  return cudaSuccess;
-}
-
-cudaError_t launch_attn_bwd(const BwdArgs& a, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(attn_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DQ_SMEM);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(attn_bwd_dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DKV_SMEM);
-  if (e != cudaSuccess) return e;
-  attn_bwd_dq_kernel<<<dim3(static_cast<unsigned>((a.n_q + BT - 1) / BT), a.H), 128, DQ_SMEM, st>>>(a);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  for (int seg = 0; seg < a.nseg; ++seg) {
-    if (!a.dk[seg]) continue;
-    attn_bwd_dkv_kernel<<<dim3(static_cast<unsigned>((a.n_k[seg] + BT - 1) / BT), a.H), 128, DKV_SMEM, st>>>(a, seg);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
-  return cudaSuccess;
-}
 
 namespace {
 

@@ -164,9 +164,6 @@ struct BwdArgs {
   Grid g;
   float scale_log2, scale;
 };
-cudaError_t launch_attn_bwd(const BwdArgs& a, cudaStream_t st);
-// dK/dV only (mma.sync kernels), for use with the tcgen05 dQ kernel
-cudaError_t launch_attn_bwd_dkv(const BwdArgs& a, cudaStream_t st);
 // dQ on tcgen05/TMEM/TMA: 128 query rows per CTA; heads packed (q_hs = n_q * 64,
 // kv_hs = n_k * 64); split scores (q_lo, k_lo) with one key segment only
 cudaError_t launch_attn_bwd_dq_tc(const BwdArgs& a, int* err, cudaStream_t st);
