@@ -164,7 +164,7 @@ GSA_API int gsa_backward(gsa_ctx *ctx,
 
 /* gsa_forward with HOST buffers: the same arguments and layouts, every tensor
  * pointer (inputs, outputs, optional sel_idx_out) in host memory.  The heads
- * are processed in up to eight chunks: the host-to-device copies of chunk i+1
+ * are processed in up to sixteen chunks: the host-to-device copies of chunk i+1
  * and the device-to-host copies of chunk i-1 overlap the layer on chunk i
  * (two extra streams of the context).  Asynchronous on `stream`: the outputs
  * are in host memory once `stream` has completed; the inputs may be reused

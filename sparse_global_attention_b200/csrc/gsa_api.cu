@@ -13,7 +13,7 @@ namespace {
 
 constexpr size_t ALIGN = 256;
 constexpr int MAX_EVENTS = 16;
-constexpr int MAX_CHUNKS = 8;          // head chunks of the host-buffer pipeline
+constexpr int MAX_CHUNKS = 16;         // head chunks of the host-buffer pipeline
 
 size_t align_up(size_t x) { return (x + ALIGN - 1) / ALIGN * ALIGN; }
 
