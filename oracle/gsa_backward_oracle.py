@@ -114,3 +114,42 @@ def backward_head(arrays, idx, d_o_img, d_o_spec, **kw):
         gr = t[n].grad
         out["d" + n] = np.zeros(t[n].shape) if gr is None else gr.numpy()
     return out
+
+
+def attention_backward_rows(q, k, v, d_o, scale, *, q_rows, k_cols, chunk=64):
+    """Gradients of O = softmax(q k^T * scale) v at selected rows and key columns,
+    in float64 numpy, for attention sizes that autograd cannot hold at once.
+
+    The closed form of the softmax-attention gradient (the same step the
+    backward of every attention of the layer takes):
+        P = softmax(S), S = q k^T * scale,  O = P v,  D_i = sum_c dO_ic O_ic,
+        dS = P o (dO v^T - D),  dq = scale dS k,  dk = scale dS^T q,  dv = P^T dO.
+    dq is returned for the query rows q_rows, dk and dv for the key columns
+    k_cols (these sum over every query, processed `chunk` rows at a time).
+    Pinned in tests/test_oracle_backward.py against torch autograd.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    d_o = np.asarray(d_o, dtype=np.float64)
+    q_rows = np.asarray(q_rows)
+    k_cols = np.asarray(k_cols)
+    row_set = {int(r): i for i, r in enumerate(q_rows)}
+    dq = np.zeros((len(q_rows), q.shape[1]))
+    dk = np.zeros((len(k_cols), k.shape[1]))
+    dv = np.zeros((len(k_cols), v.shape[1]))
+    for r0 in range(0, q.shape[0], chunk):
+        rows = slice(r0, min(r0 + chunk, q.shape[0]))
+        s = (q[rows] @ k.T) * scale
+        p = np.exp(s - s.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        o = p @ v
+        dd = (d_o[rows] * o).sum(axis=1, keepdims=True)
+        ds = p * (d_o[rows] @ v.T - dd)
+        dk += scale * ds[:, k_cols].T @ q[rows]
+        dv += p[:, k_cols].T @ d_o[rows]
+        for i in range(rows.start, rows.stop):
+            j = row_set.get(i)
+            if j is not None:
+                dq[j] = scale * ds[i - rows.start] @ k
+    return {"dq": dq, "dk": dk, "dv": dv}
