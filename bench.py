@@ -381,6 +381,22 @@ def run_b200(args, cfg, rank, world, local, dist):
         dfl = work["dense"]["flops"]
         dense = {"ms": round(dms, 2), "tflops": round(dfl / (dms / 1e3) / 1e12, 1),
                  "frac": round(dfl / (dms / 1e3) / 1e12 / tpeak, 4), "reps": 1}
+        # context only: PyTorch's own attention (its default backend) on one head of
+        # the same dense shape, bf16, no mask (this workload has no pad tokens)
+        if cfg.grid_h == cfg.pad_h and cfg.grid_w == cfg.pad_w:
+            import torch.nn.functional as tnf
+            qh, kh, vh = (t[:1].unsqueeze(0) for t in (qd, kd, vd))
+            with torch.cuda.stream(stream):
+                tnf.scaled_dot_product_attention(qh, kh, vh)
+                s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                s0.record(stream)
+                for _ in range(2):
+                    tnf.scaled_dot_product_attention(qh, kh, vh)
+                s1.record(stream)
+            torch.cuda.synchronize()
+            sms = s0.elapsed_time(s1) / 2
+            sfl = dfl / H
+            dense["torch_sdpa_one_head"] = {"ms": round(sms, 2), "tflops": round(sfl / (sms / 1e3) / 1e12, 1)}
         del qd, kd, vd, od
         torch.cuda.empty_cache()
         out = {"o_img": torch.empty_like(x["q_img"]), "o_spec": torch.empty_like(x["q_spec"])}
