@@ -74,39 +74,62 @@ __global__ void __launch_bounds__(256) rowdot_kernel(const float* do32, const __
 
 // dW_g[h][c][k] += sum over a chunk of tokens of da[t][c] q[t][k]; 256 threads,
 // 16 outputs each, tokens staged 64 at a time
-constexpr int DWG_CHUNK = 4096;
+constexpr int DWG_CHUNK = 4096;                   // tokens per CTA
+// dW_g[h] += sum over the CTA's tokens of da[t] q[t]^T: 64-token blocks staged
+// in shared memory as fp32, each thread a 4 x 4 tile of the 64 x 64 result
+// (two 16-byte shared loads per 16 FMAs), one atomic add per output at the end
 __global__ void __launch_bounds__(256) dwg_kernel(const float* da, const __nv_bfloat16* q, long long tokens,
                                                   float* dwg) {
-  __shared__ float sa[64][65];
-  __shared__ float sq[64][65];
+  __shared__ __align__(16) float sa[64][68];       // [token][channel of da]
+  __shared__ __align__(16) float sq[64][68];       // [token][channel of q]
   const int h = blockIdx.y;
   const long long t0 = static_cast<long long>(blockIdx.x) * DWG_CHUNK;
   const float* dah = da + h * tokens * D;
   const __nv_bfloat16* qh = q + h * tokens * D;
-  const int c = threadIdx.x >> 2;                 // output row (channel of da)
-  const int k0 = (threadIdx.x & 3) * 16;           // 16 columns
-  float acc[16];
+  const int tc = (threadIdx.x >> 4) * 4;           // rows tc..tc+3 of dW_g (channels of da)
+  const int tk = (threadIdx.x & 15) * 4;           // columns tk..tk+3 (channels of q)
+  float acc[4][4];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
   for (long long tb = t0; tb < t0 + DWG_CHUNK && tb < tokens; tb += 64) {
     __syncthreads();
-    for (int e = threadIdx.x; e < 64 * 64; e += 256) {
-      const int r = e >> 6, cc = e & 63;
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {                // da: 64 x 64 fp32 as float4
+      const int e = threadIdx.x + 256 * it, r = e >> 4, c4 = (e & 15) * 4;
       const bool ok = tb + r < tokens;
-      sa[r][cc] = ok ? dah[(tb + r) * D + cc] : 0.f;
-      sq[r][cc] = ok ? __bfloat162float(qh[(tb + r) * D + cc]) : 0.f;
+      const float4 v = ok ? *reinterpret_cast<const float4*>(dah + (tb + r) * D + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      *reinterpret_cast<float4*>(&sa[r][c4]) = v;
+    }
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {                // q: 64 x 64 bf16 as 8-element pieces
+      const int e = threadIdx.x + 256 * it, r = e >> 3, c8 = (e & 7) * 8;
+      const bool ok = tb + r < tokens;
+      const uint4 raw = ok ? *reinterpret_cast<const uint4*>(qh + (tb + r) * D + c8) : make_uint4(0u, 0u, 0u, 0u);
+      const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&raw);
+      *reinterpret_cast<float4*>(&sq[r][c8]) =
+          make_float4(__low2float(b[0]), __high2float(b[0]), __low2float(b[1]), __high2float(b[1]));
+      *reinterpret_cast<float4*>(&sq[r][c8 + 4]) =
+          make_float4(__low2float(b[2]), __high2float(b[2]), __low2float(b[3]), __high2float(b[3]));
     }
     __syncthreads();
-#pragma unroll 4
+#pragma unroll 8
     for (int r = 0; r < 64; ++r) {
-      const float av = sa[r][c];
+      const float4 a = *reinterpret_cast<const float4*>(&sa[r][tc]);
+      const float4 b = *reinterpret_cast<const float4*>(&sq[r][tk]);
+      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-      for (int i = 0; i < 16; ++i) acc[i] = fmaf(av, sq[r][k0 + i], acc[i]);
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
     }
   }
-  float* out = dwg + static_cast<long long>(h) * D * D + c * D + k0;
+  float* out = dwg + static_cast<long long>(h) * D * D;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) atomicAdd(out + i, acc[i]);
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) atomicAdd(out + (tc + i) * D + tk + j, acc[i][j]);
 }
 
 }  // namespace
