@@ -463,7 +463,10 @@ constexpr int SB_DST = SB_DO + 16 * 128;
 constexpr int SB_PT = SB_DST + SEL_BN * 32;
 constexpr int SB_REG = SB_PT + SEL_BN * 32;
 constexpr int SB_VAL = SB_REG + KC_MAX * 8;
-constexpr int SB_WARP = (SB_VAL + 2 * SEL_BN + 127) / 128 * 128;
+constexpr int SB_WARP = (SB_VAL + 2 * SEL_BN + 63) / 64 * 64;
+// windows (warps) per CTA of the backward: two CTAs of five warps fit the 228 KB
+// of shared memory per SM (23,104 bytes per warp; with 128-byte rounding they do not)
+constexpr int SB_WARPS = 5;
 
 // A fragments (m16 x k16) of rows [r0, r0 + 16) of a [rows][16] bf16 tile with a 32-byte pitch
 __device__ __forceinline__ void ldsm_pitch32(uint32_t base, int r0, uint32_t (&a)[4]) {
@@ -479,7 +482,7 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
 }
 
 template <int S>
-__global__ void __launch_bounds__(SEL_WARPS * 32) sel_bwd_kernel(const SelBwdArgs b) {
+__global__ void __launch_bounds__(SB_WARPS * 32) sel_bwd_kernel(const SelBwdArgs b) {
   const SelArgs& a = b.s;
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -493,7 +496,7 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) sel_bwd_kernel(const SelBwdArg
   int2* sReg = reinterpret_cast<int2*>(wbase + SB_REG);
   uint8_t* sValid = wbase + SB_VAL;
 
-  const long long win = static_cast<long long>(blockIdx.x) * SEL_WARPS + warp;
+  const long long win = static_cast<long long>(blockIdx.x) * SB_WARPS + warp;
   if (win >= static_cast<long long>(a.H) * a.R) return;      // warp-uniform
   const int h = static_cast<int>(win / a.R);
   const int r = static_cast<int>(win - static_cast<long long>(h) * a.R);
@@ -890,11 +893,11 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) sel_bwd_kernel(const SelBwdArg
 
 template <int S>
 cudaError_t launch_sel_bwd_s(const SelBwdArgs& b, cudaStream_t st) {
-  const int sm = SEL_WARPS * SB_WARP;
+  const int sm = SB_WARPS * SB_WARP;
   cudaError_t e = cudaFuncSetAttribute(sel_bwd_kernel<S>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
   if (e != cudaSuccess) return e;
   const long long w = static_cast<long long>(b.s.H) * b.s.R;
-  sel_bwd_kernel<S><<<static_cast<unsigned>((w + SEL_WARPS - 1) / SEL_WARPS), SEL_WARPS * 32, sm, st>>>(b);
+  sel_bwd_kernel<S><<<static_cast<unsigned>((w + SB_WARPS - 1) / SB_WARPS), SB_WARPS * 32, sm, st>>>(b);
   return cudaGetLastError();
 }
 
