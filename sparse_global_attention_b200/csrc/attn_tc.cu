@@ -1315,7 +1315,7 @@ void attn_tc_split(int H, long long n_q, int tiles_total, int* tiles_per_split, 
   for (long long ns = lo; ns <= maxs && ns <= 4 * lo; ++ns) {
     const long long tot = ctas * ns;
     const double eff = static_cast<double>(tot) / static_cast<double>(SMS * ((tot + SMS - 1) / SMS));
-    if (eff > best_eff + 0.02) {
+    if (eff > best_eff + 0.01) {
       best_eff = eff;
       best = ns;
     }
