@@ -731,6 +731,8 @@ struct BwdTc {
   BwdArgs b;
   int tiles0;                  // 128-key tiles of segment 0
   int tiles_total;
+  int tiles_per_split;         // dQ: key tiles per split (blockIdx.z)
+  int n_split;                 // dQ: > 1 adds each split's part to a zeroed dq
   int* err;
 };
 
@@ -804,7 +806,9 @@ __global__ void __launch_bounds__(BW_NTHREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int h = blockIdx.y;
   const int row0 = blockIdx.x * TBM;
-  const int ntile = t.tiles_total;
+  // this CTA's key tiles: split blockIdx.z of the key range
+  const int t_begin = blockIdx.z * t.tiles_per_split;
+  const int ntile = max(min(t.tiles_per_split, t.tiles_total - t_begin), 0);
 
   if (threadIdx.x == 0) {
     mbar_init(bars.q_full(), 1);
@@ -844,7 +848,7 @@ __global__ void __launch_bounds__(BW_NTHREADS, 1)
             !__all_sync(0xffffffffu, mbar_wait(bars.empty(s), ((it / L::NST) - 1) & 1, t.err)))
           break;
         long long kb;
-        const int seg = bw_seg(t, it, kb);
+        const int seg = bw_seg(t, t_begin + it, kb);
         const int y = static_cast<int>(static_cast<long long>(h) * a.n_k[seg] + kb);
         const uint32_t st = sbase + L::KV + s * L::STAGE;
         if (leader) {
@@ -932,7 +936,7 @@ __global__ void __launch_bounds__(BW_NTHREADS, 1)
       if (!ok) break;
       tc_fence_after();
       long long kb;
-      const int seg = bw_seg(t, j, kb);
+      const int seg = bw_seg(t, t_begin + j, kb);
       const int nk = a.n_k[seg];
       const int km = a.kmask[seg];
       uint32_t vm[4] = {~0u, ~0u, ~0u, ~0u};
@@ -983,12 +987,19 @@ __global__ void __launch_bounds__(BW_NTHREADS, 1)
           for (int e = 0; e < 32; e += 4) {
             float4 v = make_float4(__uint_as_float(w[e]) * a.scale, __uint_as_float(w[e + 1]) * a.scale,
                                    __uint_as_float(w[e + 2]) * a.scale, __uint_as_float(w[e + 3]) * a.scale);
-            float4* p = reinterpret_cast<float4*>(out + 32 * c + e);
-            if (a.dq_accum) {
-              const float4 o = *p;
-              v.x += o.x; v.y += o.y; v.z += o.z; v.w += o.w;
+            float* p = out + 32 * c + e;
+            if (t.n_split > 1) {
+              // key splits: each adds its part (dq was zeroed by the launcher)
+              asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"l"(p), "f"(v.x), "f"(v.y),
+                           "f"(v.z), "f"(v.w)
+                           : "memory");
+            } else {
+              if (a.dq_accum) {
+                const float4 o = *reinterpret_cast<const float4*>(p);
+                v.x += o.x; v.y += o.y; v.z += o.z; v.w += o.w;
+              }
+              *reinterpret_cast<float4*>(p) = v;
             }
-            *p = v;
           }
         }
       }
@@ -1006,7 +1017,7 @@ cudaError_t launch_dq_tc(const BwdTc& t, const CUtensorMap* maps, cudaStream_t s
   const int sm = DqLay<SPLIT>::BYTES;
   cudaError_t e = cudaFuncSetAttribute(attn_bwd_dq_tc_kernel<SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
   if (e != cudaSuccess) return e;
-  dim3 grid((t.b.n_q + TBM - 1) / TBM, t.b.H);
+  dim3 grid((t.b.n_q + TBM - 1) / TBM, t.b.H, t.n_split);
   attn_bwd_dq_tc_kernel<SPLIT><<<grid, BW_NTHREADS, sm, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5],
                                                               maps[6], maps[7], t);
   return cudaGetLastError();
@@ -1376,6 +1387,15 @@ cudaError_t launch_attn_bwd_dq_tc(const BwdArgs& b, int* err, cudaStream_t st) {
   t.tiles0 = attn_tc_tiles(b.n_k[0]);
   t.tiles_total = t.tiles0 + (b.nseg > 1 ? attn_tc_tiles(b.n_k[1]) : 0);
   t.err = err;
+  // key-range splits fill the last wave (128-row CTAs: the split rule's row count doubles);
+  // the splits add into a zeroed dq, so packed heads and an overwriting call only
+  attn_tc_split(b.H, 2LL * b.n_q, t.tiles_total, &t.tiles_per_split, &t.n_split);
+  if (b.dq_accum || b.dq_hs != static_cast<long long>(b.n_q) * D) {
+    t.tiles_per_split = t.tiles_total;
+    t.n_split = 1;
+  }
+  if (t.n_split > 1 && cudaMemsetAsync(b.dq, 0, static_cast<size_t>(H) * b.n_q * D * sizeof(float), st) != cudaSuccess)
+    return cudaErrorUnknown;
   return split ? launch_dq_tc<true>(t, maps, st) : launch_dq_tc<false>(t, maps, st);
 }
 
@@ -1395,6 +1415,8 @@ cudaError_t launch_attn_bwd_dkv_tc(const BwdArgs& b, int* err, cudaStream_t st) 
   t.b = b;
   t.tiles0 = 0;
   t.tiles_total = 0;
+  t.tiles_per_split = 0;
+  t.n_split = 1;
   t.err = err;
   for (int seg = 0; seg < b.nseg; ++seg) {
     if (!b.dk[seg]) continue;
