@@ -353,6 +353,13 @@ def run_b200(args, cfg, rank, world, local, dist):
     roof["traffic"] = read_traffic(dom, cfg.name)
     tensor_flops = sum(work[k]["flops"] for k in ("comp_attn_topk", "special", "selection", "epilogue"))
     pct_peak = tensor_flops / (ms / 1e3) / 1e12 / tpeak
+    # whole-layer roofline fraction: each launched kernel's own roofline time
+    # (the larger of FLOPs / bf16 peak and bytes / copy peak), summed, over the step time
+    roof_ms = 0.0
+    for k in kernel_ms:
+        w = work.get(k, {"flops": 0.0, "bytes": 0.0})
+        roof_ms += 1e3 * max(w["flops"] / (tpeak * 1e12), w["bytes"] / (pk["hbm_gbs"] * 1e9))
+    layer_roof = round(roof_ms / ms, 4)
 
     # ---- dense global attention of the same shape (speedup denominator) ---------
     dense = None
@@ -545,7 +552,7 @@ def run_b200(args, cfg, rank, world, local, dist):
                    "special_tokens": cfg.num_spec, "regions": cfg.num_regions,
                    "l2": "inputs 7.9 GB per GPU >> 126 MB L2: no flush between steps",
                    "parallelism": f"{world} independent replica(s), one per GPU, no collective on the data path"},
-        "roofline": roof, "pct_bf16_peak": round(pct_peak, 4),
+        "roofline": roof, "pct_bf16_peak": round(pct_peak, 4), "layer_roofline_frac": layer_roof,
         "speedup_vs_dense": (round(dense["ms"] / ms, 2) if dense else None), "dense": dense,
         "kernels": kernels, "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(), "e2e": e2e, "cpu_baseline": cpu,
