@@ -37,6 +37,8 @@ if ROOT not in sys.path:
 METRIC = "GSA layer image tokens/s at 1000 views; % of bf16 peak; speedup vs dense attn"
 UNIT = "image tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 << 20
+FLUSH_BYTES = 256 << 20
 
 # kernels of one step (names reported by gsa_get_kernel_times) and how each is graded
 TENSOR_KERNELS = {"comp_attn_topk", "special", "dense"}
@@ -302,17 +304,35 @@ def run_b200(args, cfg, rank, world, local, dist):
         raise RuntimeError(f"device status {st} during warm-up: {gsa.gsa_strerror(st)}")
 
     # ---- timed region: K steps, inputs resident in HBM ------------------------
+    # inputs far above the 126 MB L2 need no flush; smaller workloads get a 256 MB
+    # write before every step, outside each step's own pair of events
+    in_bytes = sum(t.numel() * t.element_size() for t in x.values())
+    flush = in_bytes < 4 * L2_BYTES
+    fbuf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev) if flush else None
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
-        e0.record(stream)
-        for _ in range(args.steps):
-            layer.forward(x, out=out)
-        e1.record(stream)
-        torch.cuda.synchronize()
+        if flush:
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+            for a0, a1 in evs:
+                fbuf.fill_(1)
+                a0.record(stream)
+                layer.forward(x, out=out)
+                a1.record(stream)
+            torch.cuda.synchronize()
+            step_ms = sum(a0.elapsed_time(a1) for a0, a1 in evs) / args.steps
+        else:
+            e0.record(stream)
+            for _ in range(args.steps):
+                layer.forward(x, out=out)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            step_ms = e0.elapsed_time(e1) / args.steps
     barrier()
-    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dist, dev)
+    ms = max_over_ranks(step_ms, dist, dev)
+    del fbuf
     value = throughput(world, cfg.num_img_valid, ms)
 
     # ---- per-kernel times (CUDA events recorded by the library on its stream) --
@@ -373,7 +393,7 @@ def run_b200(args, cfg, rank, world, local, dist):
         torch.cuda.empty_cache()
         qd, kd, vd = (dense_layout(x[n + "_spec"], x[n + "_img"]) for n in "qkv")
         od = torch.empty_like(qd)
-        small = gsa.GSALayer.from_workload(cfg.with_(num_frames=2))
+        small = gsa.GSALayer.from_workload(cfg.with_(num_frames=2, fixed_frames=()))   # warms the dense kernel
         small.dense(qd[:, :2 * (cfg.num_special + cfg.pad_h * cfg.pad_w)].contiguous(),
                     kd[:, :2 * (cfg.num_special + cfg.pad_h * cfg.pad_w)].contiguous(),
                     vd[:, :2 * (cfg.num_special + cfg.pad_h * cfg.pad_w)].contiguous())
@@ -550,7 +570,9 @@ def run_b200(args, cfg, rank, world, local, dist):
         "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
         "config": {"workload": workload_desc(cfg), "image_tokens": cfg.num_img_valid,
                    "special_tokens": cfg.num_spec, "regions": cfg.num_regions,
-                   "l2": "inputs 7.9 GB per GPU >> 126 MB L2: no flush between steps",
+                   "l2": (f"inputs {in_bytes / 1e9:.2f} GB per GPU >> 126 MB L2: no flush between steps" if not flush
+                          else f"inputs {in_bytes / 1e6:.0f} MB: a {FLUSH_BYTES >> 20} MB write before every step, "
+                               "outside the step's events"),
                    "parallelism": f"{world} independent replica(s), one per GPU, no collective on the data path"},
         "roofline": roof, "pct_bf16_peak": round(pct_peak, 4), "layer_roofline_frac": layer_roof,
         "speedup_vs_dense": (round(dense["ms"] / ms, 2) if dense else None), "dense": dense,
