@@ -41,7 +41,7 @@ L2_BYTES = 126 << 20
 FLUSH_BYTES = 256 << 20
 
 # kernels of one step (names reported by gsa_get_kernel_times) and how each is graded
-TENSOR_KERNELS = {"comp_attn_topk", "special", "dense"}
+TENSOR_KERNELS = {"comp_attn_topk", "special", "fixed_attn", "dense"}
 
 
 def peaks():
@@ -88,6 +88,14 @@ def algorithmic_work(cfg, kc):
     # O'_comp and the region lists; writes O_img
     w["selection_gate"] = {"flops": w["selection"]["flops"] + w["epilogue"]["flops"],
                            "bytes": 4.0 * H * slots * d * e + H * R * d * 4 + H * R * cfg.topk * 4}
+    if nfix_keys and cfg.dtype == "bf16":
+        # the fixed context runs apart: gather of its K/V (read + write), one dense attention
+        # of every image query over it (reads Q, writes the fp32 output and its LSE); the
+        # selection then attends only the selected regions and reads that output back
+        w["fixed_attn"] = {"flops": 4.0 * d * M * nfix_keys * H,
+                           "bytes": 6.0 * H * nfix_keys * d * e + H * slots * d * (e + 4) + H * slots * 4}
+        w["selection_gate"]["flops"] -= w["fixed_attn"]["flops"]
+        w["selection_gate"]["bytes"] += H * slots * (d + 1) * 4
     w["special"] = {"flops": 4.0 * d * Ms * (Ms + M) * H, "bytes": 2.0 * H * (Ms + slots) * d * e + 2.0 * H * Ms * d * e}
     w["special_merge"] = {"flops": 0.0, "bytes": 0.0}
     w["dense"] = {"flops": 4.0 * d * (M + Ms) ** 2 * H, "bytes": 4.0 * H * (slots + Ms) * d * e}

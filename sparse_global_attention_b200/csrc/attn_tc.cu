@@ -98,44 +98,68 @@ __device__ __forceinline__ int tile_seg(const AttnArgs& a, int tt, long long& kb
 }
 
 
-// validity bits of 32 consecutive keys starting at key0 (bit e = key0 + e).
-// A frame is `lead` always-valid keys (its special tokens, dense layout only)
-// and then Hp rows of Wp slots whose first Wv slots of the first Hv rows are
-// valid; the chunk is walked run by run (a handful of runs for 32 keys).
-__device__ __noinline__ uint32_t chunk_valid(int km, Grid g, int nk, long long key0) {
-  const long long lim = nk - key0;
-  const uint32_t m = lim >= 32 ? ~0u : (lim <= 0 ? 0u : ((1u << lim) - 1u));
-  if (km == MASK_NONE || m == 0u) return m;
-  const int lead = km == MASK_DENSE ? g.ns : 0;
-  const int per = lead + g.Hp * g.Wp;
-  int o = static_cast<int>(key0 % per);
-  uint32_t v = 0;
-  for (int e = 0; e < 32;) {
-    int run;
-    bool ok;
-    if (o < lead) {
-      run = lead - o;
-      ok = true;
-    } else {
-      const int q = o - lead, y = q / g.Wp, x = q - y * g.Wp;
-      if (y >= g.Hv) {
-        run = per - o;                          // pad rows up to the end of the frame
-        ok = false;
-      } else if (x < g.Wv) {
-        run = g.Wv - x;
-        ok = true;
-      } else {
-        run = g.Wp - x;
-        ok = false;
-      }
-    }
-    const int n = min(run, 32 - e);
-    if (ok) v |= (n >= 32 ? ~0u : ((1u << n) - 1u)) << e;
-    e += n;
-    o += n;
-    if (o >= per) o -= per;
+// validity bits of a 128-key tile, one word per 32-key chunk (bit e of word c
+// = key kb + 32c + e).  A frame is `lead` always-valid keys (its special tokens,
+// dense layout only) and then Hp rows of Wp slots whose first Wv slots of the
+// first Hv rows are valid.  One division places the tile's first key in its
+// frame; the tile is then walked run by run (a valid stretch of a grid row, its
+// pad columns, the pad rows, the lead), the position advancing without division.
+__device__ __noinline__ uint4 tile_valid(int km, Grid g, int nk, long long kb) {
+  uint32_t w[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const long long lim = nk - kb - 32 * c;
+    w[c] = lim >= 32 ? ~0u : (lim <= 0 ? 0u : ((1u << lim) - 1u));
   }
-  return m & v;
+  if (km != MASK_NONE && w[0] != 0u) {
+    const int lead = km == MASK_DENSE ? g.ns : 0;
+    const int per = lead + g.Hp * g.Wp;
+    int o = static_cast<int>(kb) % per;          // kb < nk: a key index of one head
+    int y = 0, x = 0;
+    if (o >= lead) {
+      y = (o - lead) / g.Wp;
+      x = (o - lead) - y * g.Wp;
+    }
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      uint32_t v = 0;
+      for (int e = 0; e < 32;) {
+        int run;
+        bool ok;
+        const bool in_rows = o >= lead && y < g.Hv;
+        if (o < lead) {
+          run = lead - o;
+          ok = true;
+        } else if (y >= g.Hv) {
+          run = per - o;                        // pad rows up to the end of the frame
+          ok = false;
+        } else if (x < g.Wv) {
+          run = g.Wv - x;
+          ok = true;
+        } else {
+          run = g.Wp - x;
+          ok = false;
+        }
+        const int n = min(run, 32 - e);
+        if (ok) v |= (n >= 32 ? ~0u : ((1u << n) - 1u)) << e;
+        e += n;
+        o += n;
+        if (o >= per) {
+          o = 0;                                // next frame
+          y = 0;
+          x = 0;
+        } else if (in_rows) {
+          x += n;                               // n <= Wp - x
+          if (x >= g.Wp) {
+            x = 0;
+            ++y;
+          }
+        }
+      }
+      w[c] &= v;
+    }
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 // c ? a : b through an explicit selp, so that chains of these over a
@@ -470,8 +494,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // key validity of the tile's four 32-key chunks (all ones unless ragged or padded)
       uint32_t vm[4] = {~0u, ~0u, ~0u, ~0u};
       if (km != MASK_NONE || kb + TBN > nk) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) vm[c] = chunk_valid(km, a.g, nk, kb + 32 * c);
+        const uint4 t4 = tile_valid(km, a.g, nk, kb);
+        vm[0] = t4.x; vm[1] = t4.y; vm[2] = t4.z; vm[3] = t4.w;
       }
       float mx = -INFINITY;
       if constexpr (!L::TOPK) {
@@ -941,8 +965,8 @@ __global__ void __launch_bounds__(BW_NTHREADS, 1)
       const int km = a.kmask[seg];
       uint32_t vm[4] = {~0u, ~0u, ~0u, ~0u};
       if (km != MASK_NONE || kb + TBN > nk) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) vm[c] = chunk_valid(km, a.g, nk, kb + 32 * c);
+        const uint4 t4 = tile_valid(km, a.g, nk, kb);
+        vm[0] = t4.x; vm[1] = t4.y; vm[2] = t4.z; vm[3] = t4.w;
       }
 #pragma unroll 1
       for (int hf = 0; hf < 2; ++hf) {

@@ -76,6 +76,10 @@ int validate(const gsa_config* c, Derived* d) {
 
 struct Layout {
   size_t comp16[3], complo[2], comp32[3], ocomp, idx, osel, part_o, part_ml, lse_c, lse_s, err, total;
+  // bf16 with fixed frames: the fixed context's keys/values packed per head, and
+  // the image queries' attention over them (output, base-2 LSE)
+  size_t kfix, vfix, ofix, lsefix;
+  long long nfix;   // fixed-context keys per head (0: none)
 };
 
 Layout make_layout(const gsa_config* c, const Derived& d) {
@@ -95,6 +99,13 @@ Layout make_layout(const gsa_config* c, const Derived& d) {
   L.lse_c = take(rows * 4);                                                  // for the backward
   L.lse_s = take(static_cast<size_t>(c->num_heads) * d.spec_per_head * 4);
   L.err = take(16);
+  const bool sel = c->variant != GSA_VARIANT_NO_SELECTION && c->variant != GSA_VARIANT_DESCRIPTOR;
+  L.nfix = (!d.fp32 && sel) ? static_cast<long long>(c->num_fixed_frames) * (c->num_special + c->grid_h * c->grid_w) : 0;
+  const size_t qrows = static_cast<size_t>(c->num_heads) * d.img_per_head;
+  L.kfix = L.nfix ? take(static_cast<size_t>(c->num_heads) * L.nfix * D * 2) : SIZE_MAX;
+  L.vfix = L.nfix ? take(static_cast<size_t>(c->num_heads) * L.nfix * D * 2) : SIZE_MAX;
+  L.ofix = L.nfix ? take(qrows * D * 4) : SIZE_MAX;
+  L.lsefix = L.nfix ? take(qrows * 4) : SIZE_MAX;
   L.total = off;
   return L;
 }
@@ -451,6 +462,7 @@ int forward_heads(gsa_ctx* c, int h0, int nh, const void* q_spec, const void* k_
   sa.H = H; sa.F = cf.num_frames; sa.R = d.R; sa.rpf = d.rpf; sa.topk = cf.topk; sa.s = cf.pool_s;
   sa.g = g; sa.scale_log2 = scale * LOG2E; sa.n_fixed = cf.num_fixed_frames;
   for (int i = 0; i < cf.num_fixed_frames; ++i) sa.fixed[i] = c->fixed[i];
+  sa.fix_o = nullptr; sa.fix_lse = nullptr;
   sa.err = err;
   EpiArgs ea;
   ea.q_img = q_img; ea.o_sel = osel; ea.o_comp = ocomp;
@@ -464,6 +476,34 @@ int forward_heads(gsa_ctx* c, int h0, int nh, const void* q_spec, const void* k_
   } else if (!d.fp32) {
     // O_sel is written only when the caller asked to keep intermediates
     if (!(c->profiling & GSA_PROFILE_KEEP_OSEL)) sa.o_sel = nullptr;
+    if (c->L.nfix > 0) {
+      // the fixed frames' tokens are keys of every window: one dense tensor-core
+      // attention of all image queries over them, merged into each window's
+      // softmax over its selected regions by the two log-sum-exps
+      const long long nfix = c->L.nfix;
+      const size_t qrows = static_cast<size_t>(d.img_per_head);
+      auto* kfix = reinterpret_cast<__nv_bfloat16*>(ws(c->L.kfix, static_cast<size_t>(nfix) * D * 2));
+      auto* vfix = reinterpret_cast<__nv_bfloat16*>(ws(c->L.vfix, static_cast<size_t>(nfix) * D * 2));
+      float* ofix = reinterpret_cast<float*>(ws(c->L.ofix, qrows * D * 4));
+      float* lsefix = reinterpret_cast<float*>(ws(c->L.lsefix, qrows * 4));
+      if (launch_fixed_gather(sa, kfix, vfix, st) != cudaSuccess) return GSA_ERR_CUDA;
+      AttnArgs a;
+      memset(&a, 0, sizeof(a));
+      a.q = reinterpret_cast<const __nv_bfloat16*>(q_img); a.q_hs = static_cast<long long>(qrows) * D;
+      a.n_q = static_cast<int>(qrows); a.q_mask = MASK_NONE;
+      a.nseg = 1;
+      a.k[0] = a.k[1] = kfix; a.v[0] = a.v[1] = vfix;
+      a.kv_hs[0] = a.kv_hs[1] = nfix * D; a.n_k[0] = a.n_k[1] = static_cast<int>(nfix);
+      a.kmask[0] = a.kmask[1] = MASK_NONE;
+      a.tiles0 = a.tiles_total = a.tiles_per_split = attn_tc_tiles(nfix); a.n_split = 1;
+      a.H = H; a.g = g; a.scale_log2 = scale * LOG2E;
+      a.o32 = ofix; a.o_hs = static_cast<long long>(qrows) * D;
+      a.lse = lsefix;
+      a.err = err;
+      if (launch_attn_tc(a, st) != cudaSuccess) return GSA_ERR_CUDA;
+      prof.mark("fixed_attn");
+      sa.fix_o = ofix; sa.fix_lse = lsefix;
+    }
     if (launch_sel_fused(sa, ea, st) != cudaSuccess) return GSA_ERR_CUDA;
     prof.mark("selection_gate");
   } else {

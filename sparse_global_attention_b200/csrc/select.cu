@@ -151,7 +151,8 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) sel_kernel_bf16(const SelArgs 
   __syncwarp();
 
   const int nk_dyn = a.topk * S * S;
-  const int nkeys = nk_dyn + a.n_fixed * (a.g.ns + a.g.Hp * a.g.Wp);
+  // the fixed context, when computed apart (a.fix_o), is merged at the end instead
+  const int nkeys = nk_dyn + (a.fix_o ? 0 : a.n_fixed * (a.g.ns + a.g.Hp * a.g.Wp));
   const int nblk = (nkeys + SEL_BN - 1) / SEL_BN;
 
   // each lane resolves one key of the block (the warp's 32, or 8 with s = 8)
@@ -311,12 +312,31 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) sel_kernel_bf16(const SelArgs 
     if (qr >= S * S) continue;
     const int y = wi * S + qr / S, x = wj * S + qr % S;
     const bool qv = y < a.g.Hv && x < a.g.Wv;
-    const float inv = (qv && l[rr] > 0.f) ? 1.f / l[rr] : 0.f;
     const long long tok = (static_cast<long long>(f) * a.g.Hp + y) * a.g.Wp + x;
+    // merge with the fixed context's attention (normalised O_fix, base-2 LSE L_fix):
+    // O = (O_fix 2^(L_fix - M) + o 2^(m sl2 - M)) / (2^(L_fix - M) + l 2^(m sl2 - M))
+    float inv = (qv && l[rr] > 0.f) ? 1.f / l[rr] : 0.f, wfix = 0.f;
+    const float* fo = nullptr;
+    if (a.fix_o && qv) {
+      const long long ft = static_cast<long long>(h) * a.F * a.g.Hp * a.g.Wp + tok;
+      const float lf = a.fix_lse[ft];
+      const float md = l[rr] > 0.f ? m[rr] * sl2 : -INFINITY;
+      const float mm = fmaxf(lf, md);
+      const float wf = ex2(lf - mm), wd = l[rr] > 0.f ? ex2(md - mm) : 0.f;
+      const float den = wf + l[rr] * wd;
+      inv = den > 0.f ? wd / den : 0.f;
+      wfix = den > 0.f ? wf / den : 0.f;
+      fo = a.fix_o + ft * D;
+    }
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt) {
       const int c = 8 * nt + 2 * t;
-      const float s0 = o[nt][2 * rr] * inv, s1 = o[nt][2 * rr + 1] * inv;
+      float s0 = o[nt][2 * rr] * inv, s1 = o[nt][2 * rr + 1] * inv;
+      if (fo) {
+        const float2 of = __ldg(reinterpret_cast<const float2*>(fo + c));
+        s0 = fmaf(of.x, wfix, s0);
+        s1 = fmaf(of.y, wfix, s1);
+      }
       if (oh) *reinterpret_cast<uint32_t*>(oh + tok * D + c) = pack_bf16(s0, s1);
       if constexpr (GATE) {
         float out0 = 0.f, out1 = 0.f;
@@ -910,6 +930,44 @@ cudaError_t launch_sel_bwd(const SelBwdArgs& b, cudaStream_t st) {
     case 4: return launch_sel_bwd_s<4>(b, st);
     default: return cudaErrorInvalidValue;
   }
+}
+
+namespace {
+// one thread per 16-byte piece of a fixed-context key or value row
+__global__ void __launch_bounds__(256) fixed_gather_kernel(const SelArgs a, __nv_bfloat16* kfix,
+                                                           __nv_bfloat16* vfix, int per_frame) {
+  const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long rows = static_cast<long long>(a.H) * a.n_fixed * per_frame;
+  if (gid >= rows * 8) return;
+  const int c = static_cast<int>(gid & 7);
+  const long long row = gid >> 3;                        // h * n_fixed * per_frame + i * per_frame + t
+  const int t = static_cast<int>(row % per_frame);
+  const long long hi = row / per_frame;
+  const int i = static_cast<int>(hi % a.n_fixed);
+  const int h = static_cast<int>(hi / a.n_fixed);
+  const int f = a.fixed[i];
+  const __nv_bfloat16 *ks, *vs;
+  if (t < a.g.ns) {
+    const long long o = ((static_cast<long long>(h) * a.F + f) * a.g.ns + t) * D;
+    ks = reinterpret_cast<const __nv_bfloat16*>(a.k_spec) + o;
+    vs = reinterpret_cast<const __nv_bfloat16*>(a.v_spec) + o;
+  } else {
+    const int u = t - a.g.ns, y = u / a.g.Wv, x = u - y * a.g.Wv;
+    const long long o = (((static_cast<long long>(h) * a.F + f) * a.g.Hp + y) * a.g.Wp + x) * D;
+    ks = reinterpret_cast<const __nv_bfloat16*>(a.k_img) + o;
+    vs = reinterpret_cast<const __nv_bfloat16*>(a.v_img) + o;
+  }
+  reinterpret_cast<uint4*>(kfix + row * D)[c] = reinterpret_cast<const uint4*>(ks)[c];
+  reinterpret_cast<uint4*>(vfix + row * D)[c] = reinterpret_cast<const uint4*>(vs)[c];
+}
+}  // namespace
+
+cudaError_t launch_fixed_gather(const SelArgs& a, __nv_bfloat16* kfix, __nv_bfloat16* vfix, cudaStream_t st) {
+  const int per_frame = a.g.ns + a.g.Hv * a.g.Wv;
+  const long long n = static_cast<long long>(a.H) * a.n_fixed * per_frame * 8;
+  if (n <= 0) return cudaSuccess;
+  fixed_gather_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(a, kfix, vfix, per_frame);
+  return cudaGetLastError();
 }
 
 }  // namespace gsa

@@ -23,9 +23,13 @@ S8_PAD_BF16 = GSAConfig("s8_pad_bf16", 2, 14, 13, 16, 16, 1, 2, 64, 8, 2, "bf16"
 S1_BF16 = GSAConfig("s1_bf16", 2, 6, 7, 6, 7, 1, 2, 64, 1, 5, "bf16")                       # R = 84 tokens
 ONE_FRAME_BF16 = GSAConfig("one_frame_bf16", 1, 12, 12, 12, 12, 3, 1, 64, 4, 3, "bf16")
 TOPK1_BF16 = GSAConfig("topk1_bf16", 4, 8, 8, 8, 8, 1, 2, 64, 2, 1, "bf16")
+# fixed context over several 128-key tiles with a ragged last one (3 x (3 + 17*17) = 876 keys),
+# 2x2 windows on a padded grid
+FIXED_TILES_BF16 = GSAConfig("fixed_tiles_bf16", 6, 17, 17, 18, 18, 3, 2, 64, 2, 6, "bf16", (0, 2, 5))
 
 SMALL = [CONFIGS["tiny_fp32"], RAGGED_BF16, MULTI_TILE_BF16, S2_BF16, PAD_VGGT_BF16,
-         NO_SPECIAL_BF16, PAD_F32, S8_BF16, S8_PAD_BF16, S1_BF16, ONE_FRAME_BF16, TOPK1_BF16]
+         NO_SPECIAL_BF16, PAD_F32, S8_BF16, S8_PAD_BF16, S1_BF16, ONE_FRAME_BF16, TOPK1_BF16,
+         FIXED_TILES_BF16]
 
 
 def _cuda_inputs(cfg, seed=0):
