@@ -226,11 +226,16 @@ __device__ __forceinline__ void apply_mask(uint32_t* v, uint32_t msk) {
   for (int e = 0; e < 32; ++e) v[e] = ((msk >> e) & 1u) ? v[e] : 0xff800000u;   // -inf
 }
 
-__device__ __forceinline__ bool is_fixed_region(const AttnArgs& a, int col) {
-  const int fr = col / a.rpf;
-  bool hit = false;
-  for (int f = 0; f < a.n_fixed; ++f) hit = hit || (a.fixed[f] == fr);
-  return hit;
+// bits of the 32 regions col0 .. col0 + 31 that lie in fixed-context frames
+// (never top-k candidates)
+__device__ __forceinline__ uint32_t fixed_bits(const AttnArgs& a, int col0) {
+  uint32_t b = 0;
+  for (int f = 0; f < a.n_fixed; ++f) {
+    const int lo = max(a.fixed[f] * a.rpf - col0, 0);
+    const int hi = min((a.fixed[f] + 1) * a.rpf - col0, 32);
+    if (hi > lo) b |= (hi - lo >= 32 ? ~0u : ((1u << (hi - lo)) - 1u)) << lo;
+  }
+  return b;
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
@@ -491,10 +496,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int seg = tile_seg(a, t_begin + j, kb);
       const int nk = a.n_k[seg];
       const int km = a.kmask[seg];
-      // key validity of the tile's four 32-key chunks (all ones unless ragged or padded)
+      // key validity of the tile's four 32-key chunks (all ones unless ragged or
+      // padded): from the segment's table when it has one (first used after the
+      // TMEM load of S, which covers the load's latency), else walked here
       uint32_t vm[4] = {~0u, ~0u, ~0u, ~0u};
       if (km != MASK_NONE || kb + TBN > nk) {
-        const uint4 t4 = tile_valid(km, a.g, nk, kb);
+        uint4 t4;
+        if constexpr (L::TOPK) {
+          t4 = tile_valid(km, a.g, nk, kb);           // regions: only a ragged last tile
+        } else {
+          const uint32_t* kbits = seg ? a.kbits[1] : a.kbits[0];
+          t4 = kbits ? __ldg(reinterpret_cast<const uint4*>(kbits) + (kb >> 7)) : tile_valid(km, a.g, nk, kb);
+        }
         vm[0] = t4.x; vm[1] = t4.y; vm[2] = t4.z; vm[3] = t4.w;
       }
       float mx = -INFINITY;
@@ -553,6 +566,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           uint32_t cb[2] = {0u, 0u};
           float hmx = -INFINITY;
           float cmx[2];
+          bool notmax[2] = {false, false};
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             const uint32_t msk = sel_if(hf, vm[2 + c], vm[c]);
@@ -563,19 +577,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (cmax > thr) {
 #pragma unroll
               for (int e = 0; e < 32; ++e) cb[c] |= (__uint_as_float(v[32 * c + e]) > thr ? 1u : 0u) << e;
+              if (a.n_fixed) {
+                // fixed-context regions are never candidates; if one of them held
+                // the chunk max, the max is no longer a candidate's value
+                const uint32_t fb = fixed_bits(a, static_cast<int>(kb) + 64 * hf + 32 * c);
+                notmax[c] = (cb[c] & fb) != 0u;
+                cb[c] &= ~fb;
+              }
             }
           }
           // rare: a score beats the current k-th; take the candidates in column
           // order through one insertion site for the whole half.  A chunk with a
           // single candidate needs no select tree: the candidate is the chunk max.
-          const bool one0 = __popc(cb[0]) == 1, one1 = __popc(cb[1]) == 1;
+          const bool one0 = __popc(cb[0]) == 1 && !notmax[0], one1 = __popc(cb[1]) == 1 && !notmax[1];
           while (cb[0] | cb[1]) {
             const bool lo = cb[0] != 0;
             const int e = lo ? __ffs(cb[0]) - 1 : 31 + __ffs(cb[1]);
             if (lo) cb[0] &= cb[0] - 1; else cb[1] &= cb[1] - 1;
             const float x = (lo ? one0 : one1) ? (lo ? cmx[0] : cmx[1]) : __uint_as_float(pick64(v, e));
             const int col = static_cast<int>(kb) + 64 * hf + e;
-            if (!(x > thr) || (a.n_fixed && is_fixed_region(a, col))) continue;
+            if (!(x > thr)) continue;
             topk_insert<KC>(ts, ti, x, col);
             thr = kth_score<KC>(ts, a.kc);
           }

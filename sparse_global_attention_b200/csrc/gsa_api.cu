@@ -1,5 +1,6 @@
 // C ABI of the GSA layer: config validation, workspace ownership, kernel
 // sequencing on the caller's stream.  See include/gsa.h for the contract.
+#include <vector>
 #include <math.h>
 #include <new>
 #include <string.h>
@@ -80,6 +81,10 @@ struct Layout {
   // the image queries' attention over them (output, base-2 LSE)
   size_t kfix, vfix, ofix, lsefix;
   long long nfix;   // fixed-context keys per head (0: none)
+  // bf16 on a padded grid: validity bits of one head's image tokens (pad slots
+  // 0), whole 128-key tiles, written once at create
+  size_t kbits;
+  size_t kbits_words;
 };
 
 Layout make_layout(const gsa_config* c, const Derived& d) {
@@ -106,6 +111,8 @@ Layout make_layout(const gsa_config* c, const Derived& d) {
   L.vfix = L.nfix ? take(static_cast<size_t>(c->num_heads) * L.nfix * D * 2) : SIZE_MAX;
   L.ofix = L.nfix ? take(qrows * D * 4) : SIZE_MAX;
   L.lsefix = L.nfix ? take(qrows * 4) : SIZE_MAX;
+  L.kbits_words = (!d.fp32 && d.pads) ? static_cast<size_t>(attn_tc_tiles(d.img_per_head)) * 4 : 0;
+  L.kbits = L.kbits_words ? take(L.kbits_words * 4) : SIZE_MAX;
   L.total = off;
   return L;
 }
@@ -231,6 +238,20 @@ int gsa_create(const gsa_config* cfg, gsa_ctx** out) {
     return GSA_ERR_OOM;
   }
   if (cudaMemset(c->ws + c->L.err, 0, 16) != cudaSuccess) { cudaFree(c->ws); delete c; return GSA_ERR_CUDA; }
+  if (c->L.kbits_words) {
+    // image-token validity of a padded grid (the same for every head)
+    std::vector<uint32_t> bits(c->L.kbits_words, 0u);
+    const long long per = static_cast<long long>(cfg->pad_h) * cfg->pad_w;
+    for (long long t = 0; t < d.img_per_head; ++t) {
+      const int o = static_cast<int>(t % per), y = o / cfg->pad_w, x = o % cfg->pad_w;
+      if (y < cfg->grid_h && x < cfg->grid_w) bits[t >> 5] |= 1u << (t & 31);
+    }
+    if (cudaMemcpy(c->ws + c->L.kbits, bits.data(), bits.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess) {
+      cudaFree(c->ws);
+      delete c;
+      return GSA_ERR_CUDA;
+    }
+  }
   for (int i = 0; i < MAX_EVENTS; ++i) {
     if (cudaEventCreate(&c->ev[i]) != cudaSuccess) {
       for (int j = 0; j < i; ++j) cudaEventDestroy(c->ev[j]);
@@ -540,6 +561,7 @@ int forward_heads(gsa_ctx* c, int h0, int nh, const void* q_spec, const void* k_
       a.v[1] = reinterpret_cast<const __nv_bfloat16*>(v_img);
       a.kv_hs[1] = ihs; a.n_k[1] = static_cast<int>(d.img_per_head);
       a.kmask[1] = d.pads ? MASK_IMG : MASK_NONE;
+      a.kbits[1] = c->at<const uint32_t>(c->L.kbits);
       a.tiles0 = d.spec_tiles0; a.tiles_total = d.spec_tiles_total;
       a.tiles_per_split = tps; a.n_split = nsplit;
       a.H = H; a.g = g; a.scale_log2 = scale * LOG2E;

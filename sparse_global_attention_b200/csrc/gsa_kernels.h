@@ -40,6 +40,10 @@ struct AttnArgs {
   long long kv_hs[2];
   int n_k[2];
   int kmask[2];              // MaskMode per segment
+  // optional per segment: key validity bits (bit e of word w = key 32 w + e of a
+  // head, zero from n_k up to the next 128-key tile), used instead of kmask
+  // (launches without the top-k)
+  const uint32_t* kbits[2];
   int guide_only;            // top-k only: S and the top-k, no P V and no output
   float* lse;                // optional [H][n_q] base-2 log-sum-exp per row (n_split == 1)
   int tiles0;                // 128-key tiles of segment 0
