@@ -85,6 +85,9 @@ struct Layout {
   // 0), whole 128-key tiles, written once at create
   size_t kbits;
   size_t kbits_words;
+  // the same for the dense layout of gsa_dense_forward (per frame: special tokens, then the grid)
+  size_t kbits_dense;
+  size_t kbits_dense_words;
 };
 
 Layout make_layout(const gsa_config* c, const Derived& d) {
@@ -113,6 +116,9 @@ Layout make_layout(const gsa_config* c, const Derived& d) {
   L.lsefix = L.nfix ? take(qrows * 4) : SIZE_MAX;
   L.kbits_words = (!d.fp32 && d.pads) ? static_cast<size_t>(attn_tc_tiles(d.img_per_head)) * 4 : 0;
   L.kbits = L.kbits_words ? take(L.kbits_words * 4) : SIZE_MAX;
+  const long long n_dense = static_cast<long long>(c->num_frames) * (c->num_special + c->pad_h * c->pad_w);
+  L.kbits_dense_words = (!d.fp32 && d.pads && n_dense < (1LL << 31)) ? static_cast<size_t>(attn_tc_tiles(n_dense)) * 4 : 0;
+  L.kbits_dense = L.kbits_dense_words ? take(L.kbits_dense_words * 4) : SIZE_MAX;
   L.total = off;
   return L;
 }
@@ -238,15 +244,22 @@ int gsa_create(const gsa_config* cfg, gsa_ctx** out) {
     return GSA_ERR_OOM;
   }
   if (cudaMemset(c->ws + c->L.err, 0, 16) != cudaSuccess) { cudaFree(c->ws); delete c; return GSA_ERR_CUDA; }
-  if (c->L.kbits_words) {
-    // image-token validity of a padded grid (the same for every head)
-    std::vector<uint32_t> bits(c->L.kbits_words, 0u);
-    const long long per = static_cast<long long>(cfg->pad_h) * cfg->pad_w;
-    for (long long t = 0; t < d.img_per_head; ++t) {
-      const int o = static_cast<int>(t % per), y = o / cfg->pad_w, x = o % cfg->pad_w;
-      if (y < cfg->grid_h && x < cfg->grid_w) bits[t >> 5] |= 1u << (t & 31);
+  for (int layout = 0; layout < 2; ++layout) {
+    // token validity of a padded grid, the same for every head: the image tokens
+    // alone (layout 0) or the dense layout, each frame's special tokens first (1)
+    const size_t words = layout ? c->L.kbits_dense_words : c->L.kbits_words;
+    if (!words) continue;
+    const int lead = layout ? cfg->num_special : 0;
+    const long long per = lead + static_cast<long long>(cfg->pad_h) * cfg->pad_w;
+    const long long n = static_cast<long long>(cfg->num_frames) * per;
+    std::vector<uint32_t> bits(words, 0u);
+    for (long long t = 0; t < n; ++t) {
+      const int o = static_cast<int>(t % per) - lead;
+      const bool ok = o < 0 || (o / cfg->pad_w < cfg->grid_h && o % cfg->pad_w < cfg->grid_w);
+      if (ok) bits[t >> 5] |= 1u << (t & 31);
     }
-    if (cudaMemcpy(c->ws + c->L.kbits, bits.data(), bits.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess) {
+    if (cudaMemcpy(c->ws + (layout ? c->L.kbits_dense : c->L.kbits), bits.data(), words * 4,
+                   cudaMemcpyHostToDevice) != cudaSuccess) {
       cudaFree(c->ws);
       delete c;
       return GSA_ERR_CUDA;
@@ -869,6 +882,7 @@ int gsa_dense_forward(gsa_ctx* c, const void* q, const void* k, const void* v, v
     a.v[0] = a.v[1] = reinterpret_cast<const __nv_bfloat16*>(v);
     a.kv_hs[0] = a.kv_hs[1] = hs; a.n_k[0] = a.n_k[1] = static_cast<int>(n);
     a.kmask[0] = a.kmask[1] = msk;
+    a.kbits[0] = a.kbits[1] = c->at<const uint32_t>(c->L.kbits_dense);
     a.tiles0 = a.tiles_total = a.tiles_per_split = attn_tc_tiles(n); a.n_split = 1;
     a.H = cf.num_heads; a.g = g; a.scale_log2 = scale_of(cf) * LOG2E;
     a.o16 = reinterpret_cast<__nv_bfloat16*>(o); a.o_hs = hs;
