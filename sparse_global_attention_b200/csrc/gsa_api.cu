@@ -79,9 +79,8 @@ struct Layout {
   size_t comp16[3], complo[2], comp32[3], ocomp, idx, osel, part_o, part_ml, lse_c, lse_s, err, total;
   // bf16 with fixed frames: the fixed context's keys/values packed per head, and
   // the image queries' attention over them (output, base-2 LSE)
-  size_t kfix, vfix, ofix, lsefix, qfix;
+  size_t kfix, vfix, ofix, lsefix;
   long long nfix;   // fixed-context keys per head (0: none)
-  long long fix_rows;   // its query rows per head: the valid tokens (qfix holds them) on a padded grid
   // bf16 on a padded grid: validity bits of one head's image tokens (pad slots
   // 0), whole 128-key tiles, written once at create
   size_t kbits;
@@ -110,9 +109,7 @@ Layout make_layout(const gsa_config* c, const Derived& d) {
   L.err = take(16);
   const bool sel = c->variant != GSA_VARIANT_NO_SELECTION && c->variant != GSA_VARIANT_DESCRIPTOR;
   L.nfix = (!d.fp32 && sel) ? static_cast<long long>(c->num_fixed_frames) * (c->num_special + c->grid_h * c->grid_w) : 0;
-  L.fix_rows = d.pads ? static_cast<long long>(c->num_frames) * c->grid_h * c->grid_w : d.img_per_head;
-  const size_t qrows = static_cast<size_t>(c->num_heads) * L.fix_rows;
-  L.qfix = (L.nfix && d.pads) ? take(qrows * D * 2) : SIZE_MAX;
+  const size_t qrows = static_cast<size_t>(c->num_heads) * d.img_per_head;
   L.kfix = L.nfix ? take(static_cast<size_t>(c->num_heads) * L.nfix * D * 2) : SIZE_MAX;
   L.vfix = L.nfix ? take(static_cast<size_t>(c->num_heads) * L.nfix * D * 2) : SIZE_MAX;
   L.ofix = L.nfix ? take(qrows * D * 4) : SIZE_MAX;
@@ -499,7 +496,7 @@ int forward_heads(gsa_ctx* c, int h0, int nh, const void* q_spec, const void* k_
   sa.H = H; sa.F = cf.num_frames; sa.R = d.R; sa.rpf = d.rpf; sa.topk = cf.topk; sa.s = cf.pool_s;
   sa.g = g; sa.scale_log2 = scale * LOG2E; sa.n_fixed = cf.num_fixed_frames;
   for (int i = 0; i < cf.num_fixed_frames; ++i) sa.fixed[i] = c->fixed[i];
-  sa.fix_o = nullptr; sa.fix_lse = nullptr; sa.fix_compact = 0;
+  sa.fix_o = nullptr; sa.fix_lse = nullptr;
   sa.err = err;
   EpiArgs ea;
   ea.q_img = q_img; ea.o_sel = osel; ea.o_comp = ocomp;
@@ -518,22 +515,15 @@ int forward_heads(gsa_ctx* c, int h0, int nh, const void* q_spec, const void* k_
       // attention of all image queries over them, merged into each window's
       // softmax over its selected regions by the two log-sum-exps
       const long long nfix = c->L.nfix;
-      const size_t qrows = static_cast<size_t>(c->L.fix_rows);
+      const size_t qrows = static_cast<size_t>(d.img_per_head);
       auto* kfix = reinterpret_cast<__nv_bfloat16*>(ws(c->L.kfix, static_cast<size_t>(nfix) * D * 2));
       auto* vfix = reinterpret_cast<__nv_bfloat16*>(ws(c->L.vfix, static_cast<size_t>(nfix) * D * 2));
       float* ofix = reinterpret_cast<float*>(ws(c->L.ofix, qrows * D * 4));
       float* lsefix = reinterpret_cast<float*>(ws(c->L.lsefix, qrows * 4));
       if (launch_fixed_gather(sa, kfix, vfix, st) != cudaSuccess) return GSA_ERR_CUDA;
-      // on a padded grid only the valid queries attend: packed first
-      const __nv_bfloat16* qf = reinterpret_cast<const __nv_bfloat16*>(q_img);
-      if (d.pads) {
-        auto* qc = reinterpret_cast<__nv_bfloat16*>(ws(c->L.qfix, qrows * D * 2));
-        if (launch_valid_rows(qf, qc, H, cf.num_frames, g, st) != cudaSuccess) return GSA_ERR_CUDA;
-        qf = qc;
-      }
       AttnArgs a;
       memset(&a, 0, sizeof(a));
-      a.q = qf; a.q_hs = static_cast<long long>(qrows) * D;
+      a.q = reinterpret_cast<const __nv_bfloat16*>(q_img); a.q_hs = static_cast<long long>(qrows) * D;
       a.n_q = static_cast<int>(qrows); a.q_mask = MASK_NONE;
       a.nseg = 1;
       a.k[0] = a.k[1] = kfix; a.v[0] = a.v[1] = vfix;
@@ -546,7 +536,7 @@ int forward_heads(gsa_ctx* c, int h0, int nh, const void* q_spec, const void* k_
       a.err = err;
       if (launch_attn_tc(a, st) != cudaSuccess) return GSA_ERR_CUDA;
       prof.mark("fixed_attn");
-      sa.fix_o = ofix; sa.fix_lse = lsefix; sa.fix_compact = d.pads ? 1 : 0;
+      sa.fix_o = ofix; sa.fix_lse = lsefix;
     }
     if (launch_sel_fused(sa, ea, st) != cudaSuccess) return GSA_ERR_CUDA;
     prof.mark("selection_gate");

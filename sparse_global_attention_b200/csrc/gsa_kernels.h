@@ -102,21 +102,16 @@ struct SelArgs {
   int n_fixed;
   int fixed[MAX_FIXED];
   // optional (bf16 fused kernel): the fixed context's attention computed apart, as
-  // the normalised output [H][rows][64] fp32 and its base-2 log-sum-exp [H][rows]
-  // (rows: F*Hv*Wv valid tokens when fix_compact, else F*Hp*Wp slots); the
-  // selection then attends only the dynamic keys and merges
+  // the normalised output [H][F*Hp*Wp][64] fp32 and its base-2 log-sum-exp
+  // [H][F*Hp*Wp]; the selection then attends only the dynamic keys and merges
   const float* fix_o;
   const float* fix_lse;
-  int fix_compact;
   int* err;
 };
 cudaError_t launch_sel(const SelArgs& a, bool fp32, cudaStream_t st);
 // the fixed frames' valid keys and values, packed per head as [H][n_fixed * (ns + Hv*Wv)][64]
 // (per fixed frame its special tokens, then its valid image tokens row-major)
 cudaError_t launch_fixed_gather(const SelArgs& a, __nv_bfloat16* kfix, __nv_bfloat16* vfix, cudaStream_t st);
-// the valid tokens of a padded grid, packed per head: dst [H][F*Hv*Wv][64] from src [H][F][Hp][Wp][64]
-cudaError_t launch_valid_rows(const __nv_bfloat16* src, __nv_bfloat16* dst, int H, int F, const Grid& g,
-                              cudaStream_t st);
 
 // ---- K4 upsample + gate + blend --------------------------------------------
 struct EpiArgs {

@@ -318,9 +318,7 @@ __global__ void __launch_bounds__(SEL_WARPS * 32) sel_kernel_bf16(const SelArgs 
     float inv = (qv && l[rr] > 0.f) ? 1.f / l[rr] : 0.f, wfix = 0.f;
     const float* fo = nullptr;
     if (a.fix_o && qv) {
-      const long long ft = a.fix_compact
-                               ? (static_cast<long long>(h) * a.F + f) * a.g.Hv * a.g.Wv + y * a.g.Wv + x
-                               : static_cast<long long>(h) * a.F * a.g.Hp * a.g.Wp + tok;
+      const long long ft = static_cast<long long>(h) * a.F * a.g.Hp * a.g.Wp + tok;
       const float lf = a.fix_lse[ft];
       const float md = l[rr] > 0.f ? m[rr] * sl2 : -INFINITY;
       const float mm = fmaxf(lf, md);
@@ -969,31 +967,6 @@ cudaError_t launch_fixed_gather(const SelArgs& a, __nv_bfloat16* kfix, __nv_bflo
   const long long n = static_cast<long long>(a.H) * a.n_fixed * per_frame * 8;
   if (n <= 0) return cudaSuccess;
   fixed_gather_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(a, kfix, vfix, per_frame);
-  return cudaGetLastError();
-}
-
-namespace {
-// one thread per 16-byte piece of a valid token's row
-__global__ void __launch_bounds__(256) valid_rows_kernel(const __nv_bfloat16* __restrict__ src,
-                                                         __nv_bfloat16* __restrict__ dst, long long rows, int Hp,
-                                                         int Wp, int Hv, int Wv) {
-  const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (gid >= rows * 8) return;
-  const int c = static_cast<int>(gid & 7);
-  const long long row = gid >> 3;                        // (h * F + f) * Hv * Wv + y * Wv + x
-  const long long hf = row / (static_cast<long long>(Hv) * Wv);
-  const int u = static_cast<int>(row - hf * Hv * Wv), y = u / Wv, x = u - y * Wv;
-  const long long s = (hf * Hp + y) * Wp + x;
-  reinterpret_cast<uint4*>(dst + row * D)[c] = __ldg(reinterpret_cast<const uint4*>(src + s * D) + c);
-}
-}  // namespace
-
-cudaError_t launch_valid_rows(const __nv_bfloat16* src, __nv_bfloat16* dst, int H, int F, const Grid& g,
-                              cudaStream_t st) {
-  const long long rows = static_cast<long long>(H) * F * g.Hv * g.Wv;
-  if (rows <= 0) return cudaSuccess;
-  valid_rows_kernel<<<static_cast<unsigned>((rows * 8 + 255) / 256), 256, 0, st>>>(src, dst, rows, g.Hp, g.Wp,
-                                                                                   g.Hv, g.Wv);
   return cudaGetLastError();
 }
 
