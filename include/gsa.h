@@ -204,9 +204,10 @@ GSA_API int gsa_get_intermediate(gsa_ctx *ctx, int which, void **dev_ptr, size_t
  *   GSA_PROFILE_TIMES      gsa_forward records CUDA events on its stream around
  *                          each kernel; gsa_get_kernel_times synchronises on the
  *                          last forward and writes up to `cap` durations in ms
- *                          (pool, compressed + top-k, selection (with the fused
- *                          upsample/gate/blend, or followed by a separate
- *                          epilogue), special, special-merge) and their names
+ *                          (pool, compressed + top-k, with fixed frames in bf16
+ *                          the fixed-context gather + attention, selection (with
+ *                          the fused upsample/gate/blend, or followed by a
+ *                          separate epilogue), special, special-merge) and their names
  *                          (static strings); it returns the number of entries
  *                          or a negative status.
  *   GSA_PROFILE_KEEP_OSEL  keep O_sel in the workspace (gsa_get_intermediate 5);
