@@ -103,9 +103,12 @@ def topk_bruteforce(scores_row: np.ndarray, cand: np.ndarray, k: int) -> np.ndar
 def topk_rows(scores: np.ndarray, cand: np.ndarray, k: int):
     """Exact top-k of every row of `scores` [n][R] over candidate columns.
 
-    Same result as topk_bruteforce row by row; it first finds the k-th best
-    value with a partition and then sorts only the columns >= that value (all
-    ties of the k-th value are kept, so the tie rule still decides).
+    Same result as topk_bruteforce row by row.  Each row is first narrowed to
+    the columns scoring at least a lower bound B of its (k+1)-th best candidate
+    score, then those columns are sorted by (score desc, index asc).  B is the
+    (k+1)-th largest of the row's block maxima (columns in 128 blocks): at least
+    k+1 blocks hold a value >= B, so at least k+1 candidates score >= B and every
+    column of the top k+1 (ties of the k-th value included) survives the cut.
     Returns (idx [n][k], gap_rel [n]) where gap_rel is
     (s_k - s_{k+1}) / max(|s_k|, 1e-30) over the candidate scores (inf when
     there is no (k+1)-th candidate).
@@ -113,20 +116,26 @@ def topk_rows(scores: np.ndarray, cand: np.ndarray, k: int):
     n, R = scores.shape
     ncand = int(cand.sum())
     assert 1 <= k <= ncand
-    s = np.where(cand[None, :], scores, NEG_INF)
+    s = scores if cand.all() else np.where(cand[None, :], scores, NEG_INF)
     out = np.empty((n, k), dtype=np.int64)
     gap = np.full(n, np.inf)
     kk = min(k + 1, ncand)
-    part = -np.partition(-s, kk - 1, axis=1)[:, :kk]   # kk best values, unordered
-    part.sort(axis=1)
-    kth = part[:, -k] if kk == k else part[:, 1]       # k-th best value
+    nb = min(128, R)
+    starts = (np.arange(nb) * R) // nb                                # nb non-empty column blocks
+    bmax = np.maximum.reduceat(s, starts, axis=1)                     # [n][nb]
+    cnt = (bmax > NEG_INF).sum(axis=1)
+    if np.all(cnt >= kk):
+        bound = -np.partition(-bmax, kk - 1, axis=1)[:, kk - 1]       # kk-th largest block max
+    else:
+        bound = np.full(n, NEG_INF)                                   # few candidate blocks: no cut
     for i in range(n):
-        cols = np.nonzero(s[i] >= kth[i])[0]
+        cols = np.nonzero(s[i] >= bound[i])[0]
+        cols = cols[s[i, cols] > NEG_INF] if bound[i] == NEG_INF else cols
         order = np.lexsort((cols, -s[i, cols]))
         out[i] = cols[order[:k]]
         if ncand > k:
-            sk = s[i, out[i, -1]]
-            sk1 = part[i, 0]
+            sk = s[i, cols[order[k - 1]]]
+            sk1 = s[i, cols[order[k]]]
             gap[i] = (sk - sk1) / max(abs(sk), 1e-30)
     return out, gap
 

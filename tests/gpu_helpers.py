@@ -2,11 +2,20 @@
 the CPU oracle on the same seeded inputs, and compare with the stated bars.
 
 Acceptance (per output tensor): bf16 configs max-abs <= 2e-2 and relative L2
-<= 1e-2; fp32 configs max-abs <= 1e-4.  Selected regions: for every
-compressed row whose oracle gap (s_k - s_{k+1}) / |s_k| exceeds 1e-3 the GPU's
-set must equal the oracle's; the outputs of every window are compared with an
-oracle run forced to the GPU's selection (identical sets where the gap rule
-applies, the GPU's valid choice elsewhere).
+<= 1e-2; fp32 configs max-abs <= 1e-4.  Selected regions, per compressed row,
+with s_k the oracle's k-th best candidate score:
+  * gap rule: where (s_k - s_{k+1}) / |s_k| exceeds 1e-3, the GPU's set equals
+    the oracle's;
+  * every other row (a near tie at the k-th place) is checked for validity:
+    every region the GPU chose scores at least s_k - tol in exact arithmetic,
+    and every candidate scoring above s_k + tol is among the GPU's choices, with
+    tol = 1e-3 |s_k| + 2^-14 |q_r| max_j |k_j|.  The second term covers the
+    on-chip guide scores' own error (the bf16 hi/lo split is accurate to about
+    2^-17 |q||k|), which can exceed 1e-3 |s_k| on rows whose k-th score is
+    close to zero;
+  * every chosen region is distinct and a candidate (not in a fixed frame).
+The outputs of every window are compared with an oracle run forced to the GPU's
+selection (identical sets where the gap rule applies, a valid choice elsewhere).
 """
 from __future__ import annotations
 
@@ -71,20 +80,42 @@ def head_arrays(x, h):
     return {k: to_f64_numpy(v[h]) for k, v in x.items()}
 
 
-def check_idx_gap_rule(gpu_idx, ora_idx, gap, rows=None):
-    """Sets equal where the oracle's k-th / (k+1)-th gap exceeds GAP.
-    Returns the number of rows checked and the number under the threshold."""
-    rows = np.arange(gpu_idx.shape[0]) if rows is None else np.asarray(rows)
-    checked = under = 0
-    for r in rows:
-        assert len(set(gpu_idx[r].tolist())) == gpu_idx.shape[1], f"row {r}: duplicate regions"
-        if gap[r] > GAP:
-            assert sorted(gpu_idx[r].tolist()) == sorted(ora_idx[r].tolist()), (
-                f"row {r}: selected regions differ (gap {gap[r]:.3e})")
-            checked += 1
-        else:
-            under += 1
-    return checked, under
+def check_index_rows(gpu_idx, scores, cand, k, qnorm, kmax, label="", verbose=True):
+    """Selected regions of every row of `scores` [n][R] (exact fp64 guide scores
+    of the rows, all candidate columns) against the oracle's top-k.
+
+    gpu_idx [n][k]; cand [R] bool; qnorm [n] = |q_r|; kmax = max_j |k_j|.
+    Rows over the 1e-3 relative gap must match the oracle's set exactly; every
+    other row must be a valid top-k within tol (see the module docstring).
+    Returns (rows checked exactly, rows checked for validity)."""
+    gpu_idx = np.asarray(gpu_idx, dtype=np.int64)
+    n = gpu_idx.shape[0]
+    ora_idx, gap = oracle.topk_rows(scores, cand, k)
+    assert gpu_idx.min() >= 0 and gpu_idx.max() < scores.shape[1], f"{label}: region index out of range"
+    assert cand[gpu_idx].all(), f"{label}: a chosen region is not a candidate"
+    srt = np.sort(gpu_idx, axis=1)
+    assert (srt[:, 1:] != srt[:, :-1]).all(), f"{label}: duplicate regions in a row"
+    exact = gap > GAP
+    bad = np.nonzero(exact & (np.sort(ora_idx, axis=1) != srt).any(axis=1))[0]
+    assert bad.size == 0, (f"{label}: selected regions differ on {bad.size} rows over the gap "
+                           f"(first row {bad[0]}, gap {gap[bad[0]]:.3e})")
+    s_k = np.take_along_axis(scores, ora_idx[:, -1:], axis=1)[:, 0]
+    tol = 1e-3 * np.abs(s_k) + 2.0 ** -14 * qnorm * kmax
+    chosen = np.take_along_axis(scores, gpu_idx, axis=1)
+    low = np.nonzero((chosen < (s_k - tol)[:, None]).any(axis=1))[0]
+    assert low.size == 0, (f"{label}: row {low[0]} chose a region scoring "
+                           f"{chosen[low[0]].min():.6g} < s_k - tol = {s_k[low[0]] - tol[low[0]]:.6g}")
+    must = scores > (s_k + tol)[:, None]              # candidates clearly above the k-th place
+    if not cand.all():
+        must &= cand[None, :]
+    hit = np.take_along_axis(must, gpu_idx, axis=1).sum(axis=1)
+    miss = np.nonzero(hit != must.sum(axis=1))[0]
+    assert miss.size == 0, f"{label}: row {miss[0]} misses a region scoring above s_k + tol"
+    under = int((~exact).sum())
+    if verbose:
+        print(f"[index] {label}: {n} rows, {n - under} over the 1e-3 gap (sets identical), "
+              f"{under} near ties ({under / max(n, 1):.1%}) checked for validity")
+    return n - under, under
 
 
 def compare_head(cfg, x, res, h, windows=None, spec_rows=None, gate_mode="learned", topk=None):
@@ -98,11 +129,12 @@ def compare_head(cfg, x, res, h, windows=None, spec_rows=None, gate_mode="learne
     nat = oracle.gsa_head(a["q_spec"], a["k_spec"], a["v_spec"], a["q_img"], a["k_img"], a["v_img"],
                           a["w_g"], **kw)
     win = nat["windows"]
-    # selected regions: valid, distinct, candidate frames only, gap rule
-    assert gidx[win].min() >= 0 and gidx[win].max() < cfg.num_regions
-    if cfg.fixed_frames:
-        assert not np.isin(gidx[win] // cfg.regions_per_frame, cfg.fixed_frames).any()
-    checked, under = check_idx_gap_rule(gidx, nat["idx"], nat["gap"], rows=win)
+    # selected regions: exact where the gap rule applies, a valid top-k elsewhere
+    cand = oracle.candidate_regions(cfg.num_frames, cfg.regions_per_frame, cfg.fixed_frames)
+    scores = nat["q_comp"][win] @ nat["k_comp"].T
+    kmax = float(np.linalg.norm(nat["k_comp"], axis=1).max())
+    checked, under = check_index_rows(gidx[win], scores, cand, k, np.linalg.norm(nat["q_comp"][win], axis=1),
+                                      kmax, label=f"{cfg.name} head {h}")
     # pooled tensors (fp32 copies are the exact means up to fp32 rounding)
     assert_close("Q_comp", res["q_comp"][h].float().cpu().numpy(), nat["q_comp"], cfg)
     assert_close("V_comp", res["v_comp"][h].float().cpu().numpy(), nat["v_comp"], cfg)

@@ -131,6 +131,31 @@ def test_topk_rows_equals_bruteforce_sort_with_ties():
     assert np.all(idx[:5] == np.nonzero(cand)[0][:k])   # ties -> lowest indices
 
 
+def test_topk_rows_wide_rows_against_bruteforce():
+    """Rows much wider than the 128 column blocks topk_rows narrows with: the
+    best values crowded into one block, exact ties at the k-th place, whole
+    blocks that are not candidates, and rows with fewer candidate blocks than
+    k+1."""
+    rng = np.random.default_rng(11)
+    n, R, k = 24, 3000, 32
+    sc = rng.integers(-50, 50, size=(n, R)).astype(np.float64)
+    sc[0, 100:140] = 1000.0 + np.arange(40) // 3             # the top 40 inside one block, with ties
+    sc[1, :] = 0.0
+    sc[1, 2000:2010] = 5.0                                   # 10 winners, then a 2990-way tie
+    sc[2] = rng.normal(size=R)
+    cand = np.ones(R, dtype=bool)
+    cand[500:900] = False                                    # whole blocks excluded
+    sparse = np.zeros(R, dtype=bool)
+    sparse[[3, 7, 2999, 1500, 1501] + list(range(40, 80))] = True   # candidates in few blocks
+    for c in (cand, sparse):
+        idx, gap = oracle.topk_rows(sc, c, k)
+        for i in range(n):
+            want = oracle.topk_bruteforce(sc[i], c, k)
+            assert list(idx[i]) == list(want)
+            rest = np.sort(sc[i, c])[::-1]
+            assert gap[i] == pytest.approx((rest[k - 1] - rest[k]) / max(abs(rest[k - 1]), 1e-30))
+
+
 def test_topk_continuous_and_scale_invariant():
     rng = np.random.default_rng(3)
     sc = rng.normal(size=(30, 200))
