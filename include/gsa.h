@@ -230,9 +230,11 @@ GSA_API const char *gsa_strerror(int code);
  * gives up after limit_us microseconds of global time (1 .. 1,000,000) and
  * records GSA_ERR_DEVICE_TIMEOUT in the context's error word.  Nothing faults
  * or hangs, and the context stays usable: gsa_get_status then returns (and
- * clears) GSA_ERR_DEVICE_TIMEOUT, and later calls run normally.  Returns
- * GSA_ERR_INVALID_ARG for a NULL context or a limit out of range,
- * GSA_ERR_CUDA if the launch fails. */
+ * clears) GSA_ERR_DEVICE_TIMEOUT, and later calls run normally.  With ctx NULL
+ * the code goes to the status word of the allocation-free calls on the
+ * current device instead (read with gsa_special_attention_noalloc_status).
+ * Returns GSA_ERR_INVALID_ARG for a limit out of range (checked before any
+ * CUDA call), GSA_ERR_CUDA if the launch fails. */
 GSA_API int gsa_debug_expire_wait(gsa_ctx *ctx, unsigned int limit_us, void *stream);
 
 /* Free the workspace and the context; NULL is accepted. */
@@ -261,15 +263,30 @@ GSA_API void gsa_destroy(gsa_ctx *ctx);
  *     calls that overlap on the GPU race, so issue them on one stream (or
  *     otherwise serialise them).
  *   - Returns GSA_ERR_UNSUPPORTED, without launching anything, when the
- *     partials (n_split * H * F * num_special * 264 bytes, n_split chosen as in
- *     gsa_forward) would exceed the array; GSA_ERR_INVALID_ARG for NULL
- *     pointers or bad sizes; GSA_ERR_CUDA if a launch fails. */
+ *     partials (256 + n_split * H * F * num_special * 264 bytes, n_split chosen
+ *     as in gsa_forward) would exceed the array; GSA_ERR_INVALID_ARG for NULL
+ *     pointers or bad sizes; GSA_ERR_CUDA if a launch fails.
+ *   - Device-side errors (a bounded wait that ran out, a failed index check)
+ *     are recorded in a status word inside the array, not returned here: read
+ *     them with gsa_special_attention_noalloc_status.  The word stays set until
+ *     read, and while it is set later calls stop early.
+ *   - On a padded grid (pad_h > grid_h or pad_w > grid_w) the kernel derives
+ *     the image keys' validity per key tile, because there is no workspace for
+ *     the per-tile validity table that gsa_forward builds at create; such
+ *     calls take longer than gsa_forward's special-token step (about 2x at 256
+ *     frames of a 37x37 grid stored as 40x40). */
 #define GSA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 GSA_API int gsa_special_attention_noalloc(const void *q_spec, const void *k_spec, const void *v_spec,
                                           const void *k_img, const void *v_img, void *o_spec,
                                           int num_heads, int num_frames, int num_special,
                                           int grid_h, int grid_w, int pad_h, int pad_w,
                                           float softmax_scale, void *stream);
+
+/* Status of the allocation-free calls on the current device: synchronises
+ * `stream`, returns the device status word (GSA_OK, GSA_ERR_DEVICE_TIMEOUT or
+ * GSA_ERR_DEVICE_BOUNDS) and clears it.  Allocates nothing.  Returns
+ * GSA_ERR_CUDA if a CUDA call fails. */
+GSA_API int gsa_special_attention_noalloc_status(void *stream);
 
 #ifdef __cplusplus
 }

@@ -21,9 +21,11 @@ GSA_GATE_LEARNED, GSA_GATE_COMP_ONLY, GSA_GATE_SEL_ONLY = 0, 1, 2
 GATE_MODES = {"learned": 0, "comp_only": 1, "sel_only": 2}
 VARIANTS = {"full": 0, "no_comp_value": 1, "no_selection": 2, "descriptor": 3}
 GSA_PROFILE_TIMES, GSA_PROFILE_KEEP_OSEL = 1, 2
+GSA_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024     # the static array of the allocation-free calls
 EXPORTED = ("gsa_create", "gsa_workspace_bytes", "gsa_forward", "gsa_dense_forward",
             "gsa_get_intermediate", "gsa_set_profiling", "gsa_get_kernel_times",
             "gsa_get_status", "gsa_strerror", "gsa_destroy", "gsa_special_attention_noalloc",
+            "gsa_special_attention_noalloc_status",
             "gsa_debug_expire_wait", "gsa_forward_host", "gsa_backward")
 
 
@@ -168,7 +170,8 @@ def gsa_get_status(ctx) -> int:
 
 def gsa_debug_expire_wait(ctx, limit_us: int, stream=None):
     """Failure-detection self-test: a device wait that runs out after limit_us
-    and records GSA_ERR_DEVICE_TIMEOUT in the context's error word."""
+    and records GSA_ERR_DEVICE_TIMEOUT in the context's error word (ctx None:
+    in the status word of the allocation-free calls on the current device)."""
     fn = load_library().gsa_debug_expire_wait
     fn.argtypes = [ctypes.c_void_p, ctypes.c_uint, ctypes.c_void_p]
     fn.restype = ctypes.c_int
@@ -182,6 +185,15 @@ def gsa_strerror(code: int) -> str:
 def gsa_destroy(ctx):
     if ctx:
         load_library().gsa_destroy(ctx)
+
+
+def gsa_special_attention_noalloc_status(stream=0) -> int:
+    """Device status word of the allocation-free calls on the current device
+    (synchronises `stream`, returns the code and clears it)."""
+    fn = load_library().gsa_special_attention_noalloc_status
+    fn.argtypes = [ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    return fn(stream or None)
 
 
 def gsa_special_attention_noalloc(q_spec, k_spec, v_spec, k_img, v_img, o_spec, num_heads,

@@ -951,9 +951,16 @@ int gsa_get_kernel_times(gsa_ctx* c, float* ms, const char** names, int cap) {
 }
 
 int gsa_debug_expire_wait(gsa_ctx* c, unsigned int limit_us, void* stream) {
-  if (!c || limit_us < 1 || limit_us > 1000000) return GSA_ERR_INVALID_ARG;
-  DeviceGuard dg(c->device);
+  if (limit_us < 1 || limit_us > 1000000) return GSA_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (!c) {
+    // no context: the status word of the allocation-free calls on the current device
+    int* word = nullptr;
+    const int rc = noalloc_status_word(&word);
+    if (rc != GSA_OK) return rc;
+    return launch_expire_wait(word, 1000ull * limit_us, st) == cudaSuccess ? GSA_OK : GSA_ERR_CUDA;
+  }
+  DeviceGuard dg(c->device);
   if (launch_expire_wait(c->at<int>(c->L.err), 1000ull * limit_us, st) != cudaSuccess) return GSA_ERR_CUDA;
   c->last_stream = st;
   return GSA_OK;

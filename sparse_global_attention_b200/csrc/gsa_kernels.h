@@ -141,6 +141,9 @@ struct AttnF32Args {
 };
 cudaError_t launch_attn_f32(const AttnF32Args& a, bool topk, cudaStream_t st);
 
+// ---- allocation-free calls: their device status word (static device memory) --
+int noalloc_status_word(int** out);
+
 // ---- failure-detection self-test ---------------------------------------------
 // one CTA waits on an mbarrier that nothing completes, gives up after limit_ns
 // of global time and records the timeout code in *err

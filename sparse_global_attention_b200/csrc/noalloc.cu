@@ -13,7 +13,12 @@
 // device current, and cached.  Make that first call before any stream capture.
 // Every call shares the array and finds the previous call's contents in it;
 // the split kernel writes every partial entry that the merge reads, so nothing
-// needs clearing except the status word.  Calls that overlap on the GPU race
+// needs clearing.  The array's first word is the device status word of these
+// calls: a kernel whose bounded wait runs out, or whose index check fails,
+// records its code there.  It starts at zero (static device memory is zero at
+// load), stays set until gsa_special_attention_noalloc_status reads and
+// clears it, and while it is set later calls stop early (as a context's
+// kernels do while its error word is set).  Calls that overlap on the GPU race
 // on the array: serialise them (for example, one stream).
 #include <mutex>
 #include <string.h>
@@ -48,6 +53,28 @@ int scratch_address(void** out) {
 
 }  // namespace
 
+namespace gsa {
+// the status word of the allocation-free calls on the current device
+int noalloc_status_word(int** out) {
+  void* base = nullptr;
+  const int rc = scratch_address(&base);
+  if (rc != GSA_OK) return rc;
+  *out = static_cast<int*>(base);
+  return GSA_OK;
+}
+}  // namespace gsa
+
+extern "C" int gsa_special_attention_noalloc_status(void* stream) {
+  int* word = nullptr;
+  int rc = noalloc_status_word(&word);
+  if (rc != GSA_OK) return rc;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return GSA_ERR_CUDA;
+  int code = 0;
+  if (cudaMemcpy(&code, word, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return GSA_ERR_CUDA;
+  if (code != 0 && cudaMemset(word, 0, sizeof(int)) != cudaSuccess) return GSA_ERR_CUDA;
+  return code;
+}
+
 extern "C" int gsa_special_attention_noalloc(const void* q_spec, const void* k_spec, const void* v_spec,
                                              const void* k_img, const void* v_img, void* o_spec,
                                              int num_heads, int num_frames, int num_special, int grid_h,
@@ -80,7 +107,6 @@ extern "C" int gsa_special_attention_noalloc(const void* q_spec, const void* k_s
   int* err = reinterpret_cast<int*>(b);
   float* part_o = reinterpret_cast<float*>(b + STATUS_BYTES);
   float* part_ml = part_o + rows * D;
-  if (cudaMemsetAsync(err, 0, sizeof(int), st) != cudaSuccess) return GSA_ERR_CUDA;
 
   const float scale = softmax_scale > 0.f ? softmax_scale : 0.125f;   // 1/sqrt(64)
   Grid g;

@@ -46,16 +46,26 @@ def test_fp32_contexts_keep_the_fixed_context_in_the_selection():
 
 
 def test_traffic_record_is_tied_to_the_sources(tmp_path, monkeypatch):
-    """A traffic figure is used only while the recorded source hash matches."""
+    """A traffic figure is used only while the recorded source hash matches; a
+    record of a smaller workload is scaled by the ratio of compulsory bytes."""
     prof = tmp_path / "profiles"
     prof.mkdir()
-    sha = bench.kernel_source_sha()
+    sha = "abcdef123456"
     (prof / "ncu_traffic.txt").write_text(
         "# kernel workload bytes source_sha\n"
         f"comp_attn_topk pi3_f1000 123 {sha}\n"
-        "comp_attn_topk pi3_f128 456 000000000000\n")
+        "comp_attn_topk pi3_f128 456 000000000000\n"
+        f"pool pi3_f128 1000 {sha}\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    monkeypatch.setattr(bench, "kernel_source_sha", lambda: sha)
-    assert bench.read_traffic("comp_attn_topk", "pi3_f1000") == 123.0
-    assert bench.read_traffic("comp_attn_topk", "pi3_f128") is None
-    assert bench.read_traffic("special", "pi3_f1000") is None
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda kernel="": sha)
+    assert bench.read_traffic("comp_attn_topk", "pi3_f1000")[0] == 123.0
+    assert bench.read_traffic("comp_attn_topk", "pi3_f128")[0] is None
+    assert bench.read_traffic("special", "pi3_f1000")[0] is None
+    b, note = bench.read_traffic("pool", "pi3_f1000", {"pi3_f128": 10.0, "pi3_f1000": 78.0})
+    assert b == pytest.approx(7800.0) and "scaled" in note
+    assert bench.read_traffic("pool", "pi3_f1000")[0] is None
+
+
+def test_each_kernel_hashes_its_own_sources():
+    assert bench.kernel_source_sha("pool") != bench.kernel_source_sha("comp_attn_topk")
+    assert bench.kernel_source_sha("special") == bench.kernel_source_sha("comp_attn_topk")
