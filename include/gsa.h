@@ -46,7 +46,7 @@ extern "C" {
 #define GSA_ERR_SHAPE          2  /* grid not divisible by pool_s, head_dim != 64,
                                      topk outside [1, candidates], region with no
                                      valid token                                      */
-#define GSA_ERR_UNSUPPORTED    3  /* valid but not implemented (e.g. topk > 64)       */
+#define GSA_ERR_UNSUPPORTED    3  /* valid but not implemented (e.g. topk > 128)      */
 #define GSA_ERR_OOM            4  /* workspace allocation failed                      */
 #define GSA_ERR_CUDA           5  /* a CUDA runtime call failed                       */
 #define GSA_ERR_DEVICE_TIMEOUT 6  /* a bounded device-side wait ran out               */
@@ -63,8 +63,9 @@ extern "C" {
 #define GSA_GATE_COMP_ONLY 1
 #define GSA_GATE_SEL_ONLY  2
 
-/* maximum top-k and maximum number of fixed-context frames */
-#define GSA_MAX_TOPK         64
+/* maximum top-k and maximum number of fixed-context frames; top-k above 64
+ * needs bf16 and pool_s = 4 (the notes' test-time top-128, section "测试时自适应") */
+#define GSA_MAX_TOPK         128
 #define GSA_MAX_FIXED_FRAMES 16
 
 /* Layer variants of the notes' ablation study ("消融实验", rows (1) and (2)).
@@ -102,7 +103,8 @@ typedef struct {
     int num_heads;         /* H >= 1                                              */
     int head_dim;          /* must be 64                                          */
     int pool_s;            /* s in {1, 2, 4, 8}                                   */
-    int topk;              /* regions per compressed query, 1..min(64, candidates) */
+    int topk;              /* regions per compressed query, 1..min(128, candidates);
+                              above 64 only bf16 with pool_s = 4                  */
     int dtype;             /* GSA_BF16 or GSA_FP32                                */
     const int *fixed_frames; /* VGGT fixed global context frames (copied at
                               create); NULL with num_fixed_frames = 0 for pi^3   */
@@ -150,7 +152,7 @@ GSA_API int gsa_forward(gsa_ctx *ctx,
  * dq/dk/dv_img [H][F][pad_h][pad_w][64] (0 on pads), dq/dk/dv_spec
  * [H][F][num_special][64] (unused when num_special = 0), dw_g [H][64][64]
  * (0 when the gate is forced).  bf16 contexts of the full layer with
- * pool_s <= 4 only (GSA_ERR_UNSUPPORTED otherwise); allocates a scratch of
+ * pool_s <= 4 and topk <= 64 only (GSA_ERR_UNSUPPORTED otherwise); allocates a scratch of
  * about 5 x H x R x 256 bytes plus one float per image-token channel on first
  * use (GSA_ERR_OOM if that fails), freed by gsa_destroy.  Asynchronous on
  * `stream`. */

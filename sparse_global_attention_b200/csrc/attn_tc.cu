@@ -318,7 +318,10 @@ __device__ __forceinline__ void topk_insert(float (&ts)[KC > 0 ? KC : 1], int (&
   }
 }
 
-template <int KC, bool GO>
+// EX (top-k beyond one list, passes after the first): columns at or ahead of the
+// previous pass's last selection (a.excl_s / a.excl_i) in the order (score desc,
+// index asc) are not candidates, so the pass continues the sorted selection.
+template <int KC, bool GO, bool EX = false>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qlo,
                    const __grid_constant__ CUtensorMap tm_k0, const __grid_constant__ CUtensorMap tm_v0,
@@ -488,6 +491,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       ti[p] = -1;
     }
     bool ok = true;
+    float ex_s = INFINITY;                            // EX: the previous pass's last selection
+    int ex_i = -1;
+    if constexpr (EX) {
+      if (row < a.n_q) {
+        ex_s = a.excl_s[static_cast<long long>(h) * a.n_q + row];
+        ex_i = a.excl_i[static_cast<long long>(h) * a.n_q + row];
+      }
+    }
     for (int j = 0; j < ntile; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(bars.s_full(qi), j & 1, a.err));
       if (!ok) break;
@@ -583,6 +594,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const uint32_t fb = fixed_bits(a, static_cast<int>(kb) + 64 * hf + 32 * c);
                 notmax[c] = (cb[c] & fb) != 0u;
                 cb[c] &= ~fb;
+              }
+              if constexpr (EX) {
+                if (cmax >= ex_s) {
+                  // an earlier pass took these: score above its last, or equal at a lower index
+                  const int col0 = static_cast<int>(kb) + 64 * hf + 32 * c;
+#pragma unroll 1
+                  for (int e = 0; e < 32; ++e) {
+                    const float x = __uint_as_float(v[32 * c + e]);
+                    if (x > ex_s || (x == ex_s && col0 + e <= ex_i)) cb[c] &= ~(1u << e);
+                  }
+                  notmax[c] = true;
+                }
               }
             }
           }
@@ -699,13 +722,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         *reinterpret_cast<float2*>(a.part_ml + pr * 2) = make_float2(m, l);
       }
       if constexpr (L::TOPK) {
-        const long long base = (static_cast<long long>(h) * a.n_q + row) * a.kc;
+        const long long base = (static_cast<long long>(h) * a.n_q + row) * a.cand_stride + a.cand_off;
 #pragma unroll
         for (int p = 0; p < KC; ++p) {
           if (p < a.kc) {
             a.cand[base + p] = ti[p];
             if (a.cand_user) a.cand_user[base + p] = ti[p];
           }
+        }
+        if (a.last_s) {
+          // the last selection of this pass, where the next pass continues
+          a.last_s[static_cast<long long>(h) * a.n_q + row] = kth_score<KC>(ts, a.kc);
+          int li = ti[KC - 1];
+#pragma unroll
+          for (int p = 0; p < KC; ++p) li = p == a.kc - 1 ? ti[p] : li;
+          a.last_i[static_cast<long long>(h) * a.n_q + row] = li;
         }
       }
     }
@@ -747,13 +778,13 @@ bool make_map(CUtensorMap* m, const void* base, long long rows) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int KC, bool GO>
+template <int KC, bool GO, bool EX = false>
 cudaError_t launch_kc(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t st) {
   const int sm = Lay<KC, GO>::BYTES;
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<KC, GO>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<KC, GO, EX>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
   if (e != cudaSuccess) return e;
   dim3 grid((a.n_q + 2 * TBM - 1) / (2 * TBM), a.n_split, a.H);
-  attn_tc_kernel<KC, GO><<<grid, NTHREADS, sm, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], a);
+  attn_tc_kernel<KC, GO, EX><<<grid, NTHREADS, sm, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], a);
   return cudaGetLastError();
 }
 
@@ -1399,10 +1430,10 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
   maps[6] = maps[2];
   if (a.kc > 0 && !make_map(&maps[6], a.k_lo, H * a.n_k[0])) return cudaErrorInvalidValue;
   if (a.kc == 0) return launch_kc<0, false>(a, maps, st);
+  if (a.excl_s) return (a.guide_only && a.kc <= 32) ? launch_kc<32, true, true>(a, maps, st) : cudaErrorInvalidValue;
   if (a.kc <= 8) return launch_kc2<8>(a, maps, st);
   if (a.kc <= 16) return launch_kc2<16>(a, maps, st);
   if (a.kc <= 32) return launch_kc2<32>(a, maps, st);
-  if (a.kc <= 64) return launch_kc2<64>(a, maps, st);
   return cudaErrorInvalidValue;
 }
 

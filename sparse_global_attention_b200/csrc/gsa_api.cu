@@ -63,6 +63,8 @@ int validate(const gsa_config* c, Derived* d) {
   d->ncand = d->R - c->num_fixed_frames * d->rpf;
   if (c->topk > d->ncand) return GSA_ERR_SHAPE;
   if (c->topk > GSA_MAX_TOPK) return GSA_ERR_UNSUPPORTED;
+  // beyond 64 regions only the bf16 tensor-core selection (4 x 4 windows) takes the list
+  if (c->topk > 64 && (c->dtype != GSA_BF16 || s != 4)) return GSA_ERR_UNSUPPORTED;
   d->kc = c->topk;
   d->fp32 = c->dtype == GSA_FP32;
   d->pads = c->pad_h != c->grid_h || c->pad_w != c->grid_w;
@@ -77,6 +79,7 @@ int validate(const gsa_config* c, Derived* d) {
 
 struct Layout {
   size_t comp16[3], complo[2], comp32[3], ocomp, idx, osel, part_o, part_ml, lse_c, lse_s, err, total;
+  size_t last_s, last_i;
   // bf16 with fixed frames: the fixed context's keys/values packed per head, and
   // the image queries' attention over them (output, base-2 LSE)
   size_t kfix, vfix, ofix, lsefix;
@@ -88,7 +91,17 @@ struct Layout {
   // the same for the dense layout of gsa_dense_forward (per frame: special tokens, then the grid)
   size_t kbits_dense;
   size_t kbits_dense_words;
+  // bf16 selection on tensor cores (s = 4): window order of the groups (written
+  // once at create), and per forward the union of each group's selected regions
+  size_t winof, uni, ucnt;
+  int ngroups;
 };
+
+// the tensor-core selection serves bf16 contexts with 4 x 4 windows that have a selection branch
+bool sel_on_tc(const gsa_config* c, const Derived& d) {
+  const bool sel = c->variant == GSA_VARIANT_FULL || c->variant == GSA_VARIANT_NO_COMP_VALUE;
+  return sel && !d.fp32 && c->pool_s == 4 && c->topk * SEL_GROUP <= SEL_UNION_MAX;
+}
 
 Layout make_layout(const gsa_config* c, const Derived& d) {
   Layout L;
@@ -105,6 +118,10 @@ Layout make_layout(const gsa_config* c, const Derived& d) {
   L.part_o = take(sp * D * 4);
   L.part_ml = take(sp * 2 * 4);
   L.lse_c = take(rows * 4);                                                  // for the backward
+  // top-k beyond one 32-entry list: each row's last selection of a pass, where the next pass continues
+  const bool multi = !d.fp32 && c->topk > 32;
+  L.last_s = multi ? take(rows * 4) : SIZE_MAX;
+  L.last_i = multi ? take(rows * 4) : SIZE_MAX;
   L.lse_s = take(static_cast<size_t>(c->num_heads) * d.spec_per_head * 4);
   L.err = take(16);
   const bool sel = c->variant != GSA_VARIANT_NO_SELECTION && c->variant != GSA_VARIANT_DESCRIPTOR;
@@ -119,6 +136,10 @@ Layout make_layout(const gsa_config* c, const Derived& d) {
   const long long n_dense = static_cast<long long>(c->num_frames) * (c->num_special + c->pad_h * c->pad_w);
   L.kbits_dense_words = (!d.fp32 && d.pads && n_dense < (1LL << 31)) ? static_cast<size_t>(attn_tc_tiles(n_dense)) * 4 : 0;
   L.kbits_dense = L.kbits_dense_words ? take(L.kbits_dense_words * 4) : SIZE_MAX;
+  L.ngroups = sel_on_tc(c, d) ? sel_group_count(d.R) : 0;
+  L.winof = L.ngroups ? take(static_cast<size_t>(d.R) * 4) : SIZE_MAX;
+  L.uni = L.ngroups ? take(static_cast<size_t>(c->num_heads) * L.ngroups * SEL_GROUP * c->topk * 8) : SIZE_MAX;
+  L.ucnt = L.ngroups ? take(static_cast<size_t>(c->num_heads) * L.ngroups * 4) : SIZE_MAX;
   L.total = off;
   return L;
 }
@@ -260,6 +281,15 @@ int gsa_create(const gsa_config* cfg, gsa_ctx** out) {
     }
     if (cudaMemcpy(c->ws + (layout ? c->L.kbits_dense : c->L.kbits), bits.data(), words * 4,
                    cudaMemcpyHostToDevice) != cudaSuccess) {
+      cudaFree(c->ws);
+      delete c;
+      return GSA_ERR_CUDA;
+    }
+  }
+  if (c->L.ngroups) {
+    std::vector<int> order(static_cast<size_t>(d.R));
+    sel_group_order(cfg->num_frames, cfg->pad_h / cfg->pool_s, cfg->pad_w / cfg->pool_s, order.data());
+    if (cudaMemcpy(c->ws + c->L.winof, order.data(), order.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess) {
       cudaFree(c->ws);
       delete c;
       return GSA_ERR_CUDA;
@@ -465,13 +495,32 @@ int forward_heads(gsa_ctx* c, int h0, int nh, const void* q_spec, const void* k_
     a.tiles0 = a.tiles_total = a.tiles_per_split = attn_tc_tiles(d.R); a.n_split = 1;
     a.H = H; a.g = g; a.scale_log2 = scale * LOG2E;
     a.o32 = ocomp; a.o_hs = rhs;
-    a.kc = no_sel ? 0 : d.kc; a.cand = idx; a.cand_user = sel_idx_out;
+    // the top-k runs in passes of at most 32 regions per row: the first pass is fused
+    // with the attention, each later pass is a guide-only launch that continues the
+    // sorted selection after the previous pass's last entry of the row
+    const int kt = no_sel ? 0 : d.kc;
+    a.kc = kt < 32 ? kt : 32; a.cand = idx; a.cand_user = sel_idx_out;
+    a.cand_stride = kt; a.cand_off = 0;
+    float* last_s = reinterpret_cast<float*>(ws(c->L.last_s, static_cast<size_t>(d.R) * 4));
+    int* last_i = reinterpret_cast<int*>(ws(c->L.last_i, static_cast<size_t>(d.R) * 4));
+    if (kt > 32) { a.last_s = last_s; a.last_i = last_i; }
     a.guide_only = cf.variant == GSA_VARIANT_NO_COMP_VALUE ? 1 : 0;
     a.lse = reinterpret_cast<float*>(ws(c->L.lse_c, static_cast<size_t>(d.R) * 4));
     a.rpf = d.rpf; a.n_fixed = cf.num_fixed_frames;
     for (int i = 0; i < cf.num_fixed_frames; ++i) a.fixed[i] = c->fixed[i];
     a.err = err;
     if (launch_attn_tc(a, st) != cudaSuccess) return GSA_ERR_CUDA;
+    for (int off0 = 32; off0 < kt; off0 += 32) {
+      AttnArgs b = a;
+      b.guide_only = 1;
+      b.kc = kt - off0 < 32 ? kt - off0 : 32;
+      b.cand_off = off0;
+      b.excl_s = last_s; b.excl_i = last_i;          // read and rewritten row by row
+      b.last_s = off0 + 32 < kt ? last_s : nullptr;
+      b.last_i = off0 + 32 < kt ? last_i : nullptr;
+      b.o32 = nullptr; b.lse = nullptr;
+      if (launch_attn_tc(b, st) != cudaSuccess) return GSA_ERR_CUDA;
+    }
   } else {
     AttnF32Args a;
     memset(&a, 0, sizeof(a));
@@ -538,7 +587,31 @@ int forward_heads(gsa_ctx* c, int h0, int nh, const void* q_spec, const void* k_
       prof.mark("fixed_attn");
       sa.fix_o = ofix; sa.fix_lse = lsefix;
     }
-    if (launch_sel_fused(sa, ea, st) != cudaSuccess) return GSA_ERR_CUDA;
+    if (c->L.ngroups) {
+      // groups of 8 neighbouring windows on the tensor cores: the union of their
+      // regions, then one CTA per group
+      SelTcArgs ta;
+      memset(&ta, 0, sizeof(ta));
+      ta.q_img = q_img; ta.k_img = k_img; ta.v_img = v_img; ta.w_g = w_g;
+      ta.idx = idx;
+      ta.win_of = c->at<const int>(c->L.winof);
+      ta.NG = c->L.ngroups;
+      ta.topk = cf.topk;
+      ta.emax = SEL_GROUP * cf.topk;
+      ta.uni = reinterpret_cast<uint2*>(ws(c->L.uni, static_cast<size_t>(ta.NG) * ta.emax * 8));
+      ta.ucnt = reinterpret_cast<int*>(ws(c->L.ucnt, static_cast<size_t>(ta.NG) * 4));
+      ta.o_comp = ocomp; ta.fix_o = sa.fix_o; ta.fix_lse = sa.fix_lse;
+      ta.o_img = static_cast<__nv_bfloat16*>(o_img);
+      ta.o_sel = static_cast<__nv_bfloat16*>(sa.o_sel);
+      ta.H = H; ta.F = cf.num_frames; ta.R = d.R; ta.rpf = d.rpf; ta.rx = cf.pad_w / cf.pool_s;
+      ta.g = g; ta.scale_log2 = scale * LOG2E; ta.gate_mode = gate;
+      ta.err = err;
+      if (launch_sel_union(ta, st) != cudaSuccess) return GSA_ERR_CUDA;
+      prof.mark("sel_union");
+      if (launch_sel_tc(ta, st) != cudaSuccess) return GSA_ERR_CUDA;
+    } else if (launch_sel_fused(sa, ea, st) != cudaSuccess) {
+      return GSA_ERR_CUDA;
+    }
     prof.mark("selection_gate");
   } else {
     if (launch_sel(sa, d.fp32, st) != cudaSuccess) return GSA_ERR_CUDA;
@@ -729,7 +802,7 @@ int gsa_backward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void*
   const bool spec = cf.num_special > 0;
   if (spec && (!q_spec || !k_spec || !v_spec || !o_spec || !d_o_spec || !dq_spec || !dk_spec || !dv_spec))
     return GSA_ERR_INVALID_ARG;
-  if (d.fp32 || cf.variant != GSA_VARIANT_FULL || cf.pool_s > 4) return GSA_ERR_UNSUPPORTED;
+  if (d.fp32 || cf.variant != GSA_VARIANT_FULL || cf.pool_s > 4 || cf.topk > 64) return GSA_ERR_UNSUPPORTED;
   const int gate = effective_gate(cf);
   if (gate == GSA_GATE_LEARNED && !w_g) return GSA_ERR_INVALID_ARG;
   if (cf.num_fixed_frames > 0 && !spec) return GSA_ERR_INVALID_ARG;

@@ -59,9 +59,17 @@ struct AttnArgs {
   float* part_o;             // [n_split][H][n_q][64] unnormalised
   float* part_ml;            // [n_split][H][n_q][2]  (running max in raw score units, sum)
   // streaming top-k of the raw scores (compressed branch only)
-  int kc;                    // regions kept per row (the top-k)
-  int* cand;                 // [H][n_q][kc] region indices, best first
-  int* cand_user;            // optional copy for the caller
+  int kc;                    // regions kept per row by this launch (<= 32)
+  int* cand;                 // [H][n_q][cand_stride] region indices, best first, this launch's
+  int* cand_user;            //   kc of them from column cand_off; cand_user: optional copy
+  int cand_stride, cand_off;
+  // top-k beyond one launch's list: the launch continues the selection after the
+  // previous launch's last entry per row (excl_s score, excl_i region; guide-only
+  // launches only), and writes its own last entry to last_s / last_i if set
+  const float* excl_s;
+  const int* excl_i;
+  float* last_s;
+  int* last_i;
   int rpf;                   // regions per frame
   int n_fixed;
   int fixed[MAX_FIXED];      // frames excluded from the candidates
@@ -112,6 +120,41 @@ cudaError_t launch_sel(const SelArgs& a, bool fp32, cudaStream_t st);
 // the fixed frames' valid keys and values, packed per head as [H][n_fixed * (ns + Hv*Wv)][64]
 // (per fixed frame its special tokens, then its valid image tokens row-major)
 cudaError_t launch_fixed_gather(const SelArgs& a, __nv_bfloat16* kfix, __nv_bfloat16* vfix, cudaStream_t st);
+
+// ---- K3 + K4 on tcgen05 (bf16, s = 4): groups of SEL_GROUP neighbouring windows
+// (8 x 16 queries = one 128-row MMA tile) attend to the union of their selected
+// regions, each row masked to its own window's regions --------------------------
+constexpr int SEL_GROUP = 8;
+constexpr int SEL_UNION_MAX = 1024;          // SEL_GROUP * top-k <= this (top-k <= 128)
+struct SelTcArgs {
+  const void* q_img;         // [H][F][Hp][Wp][64] bf16
+  const void* k_img;
+  const void* v_img;
+  const void* w_g;           // [H][64][64] bf16 (gate_mode 0)
+  const int* idx;            // [H][R][topk] selected regions
+  const int* win_of;         // [R] window at each group position (sel_group_order)
+  uint2* uni;                // [H][NG][emax] union entries: x region, y = (token bits << 16) | window bits
+  int* ucnt;                 // [H][NG] distinct regions per group
+  int emax;                  // SEL_GROUP * topk
+  int NG;                    // groups per head
+  int topk;
+  const float* o_comp;       // O'_comp [H][R][64] fp32
+  const float* fix_o;        // optional fixed-context attention [H][F*Hp*Wp][64] fp32 and its
+  const float* fix_lse;      //   base-2 log-sum-exp [H][F*Hp*Wp]
+  __nv_bfloat16* o_img;      // [H][F][Hp][Wp][64]
+  __nv_bfloat16* o_sel;      // optional [H][F][Hp][Wp][64]
+  int H, F, R, rpf, rx;      // rx = Wp / 4 windows per region row
+  Grid g;
+  float scale_log2;
+  int gate_mode;             // 0 g = sigmoid(W_g q), 1 g = 1, 2 g = 0
+  int* err;
+};
+int sel_group_count(int R);
+// group positions -> windows: per frame, row pairs top to bottom, walking the
+// columns alternately left to right and back (win_of has F * rows * cols entries)
+void sel_group_order(int F, int rows, int cols, int* win_of);
+cudaError_t launch_sel_union(const SelTcArgs& a, cudaStream_t st);
+cudaError_t launch_sel_tc(const SelTcArgs& a, cudaStream_t st);
 
 // ---- K4 upsample + gate + blend --------------------------------------------
 struct EpiArgs {

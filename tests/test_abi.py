@@ -37,7 +37,9 @@ def _cfg(**kw):
     (dict(pool_s=3), 3),                          # unsupported pool size
     (dict(grid_h=9), 2),                          # grid not divisible by s
     (dict(topk=0), 1),
-    (dict(topk=65, num_frames=64), 3),            # above the supported maximum
+    (dict(topk=65, num_frames=64), 3),            # above 64: fp32 keeps the 64-entry list
+    (dict(topk=100, num_frames=64, dtype="bf16"), 3),                      # above 64 with s = 2
+    (dict(topk=129, num_frames=64, dtype="bf16", pool_s=4), 3),            # above the maximum of 128
     (dict(topk=17, num_frames=1), 2),             # more than the 16 regions
     (dict(pad_h=10, grid_h=7), 2),                # a region row with no valid token
     (dict(pad_h=6, grid_h=8), 2),                 # pad smaller than the grid
@@ -54,6 +56,11 @@ def test_invalid_configs_are_rejected_on_the_host(kw, code):
     cfg = _cfg(**kw)
     assert gsa.gsa_create_status(cfg) == code
     assert gsa.gsa_workspace_bytes(cfg) == 0
+
+
+def test_top128_is_accepted_for_bf16_4x4_windows():
+    cfg = _cfg(topk=128, num_frames=64, dtype="bf16", pool_s=4)
+    assert gsa.gsa_workspace_bytes(cfg) > 0
 
 
 def test_workspace_bytes_of_named_workloads():

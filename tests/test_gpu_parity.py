@@ -23,13 +23,16 @@ S8_PAD_BF16 = GSAConfig("s8_pad_bf16", 2, 14, 13, 16, 16, 1, 2, 64, 8, 2, "bf16"
 S1_BF16 = GSAConfig("s1_bf16", 2, 6, 7, 6, 7, 1, 2, 64, 1, 5, "bf16")                       # R = 84 tokens
 ONE_FRAME_BF16 = GSAConfig("one_frame_bf16", 1, 12, 12, 12, 12, 3, 1, 64, 4, 3, "bf16")
 TOPK1_BF16 = GSAConfig("topk1_bf16", 4, 8, 8, 8, 8, 1, 2, 64, 2, 1, "bf16")
+# 4 x 4 windows with one region each, and a head count / window count that leaves
+# ragged groups of the tensor-core selection (R = 3 x 9 = 27, groups of 8)
+TOPK1_S4_BF16 = GSAConfig("topk1_s4_bf16", 3, 12, 12, 12, 12, 1, 3, 64, 4, 1, "bf16")
 # fixed context over several 128-key tiles with a ragged last one (3 x (3 + 17*17) = 876 keys),
 # 2x2 windows on a padded grid
 FIXED_TILES_BF16 = GSAConfig("fixed_tiles_bf16", 6, 17, 17, 18, 18, 3, 2, 64, 2, 6, "bf16", (0, 2, 5))
 
 SMALL = [CONFIGS["tiny_fp32"], RAGGED_BF16, MULTI_TILE_BF16, S2_BF16, PAD_VGGT_BF16,
          NO_SPECIAL_BF16, PAD_F32, S8_BF16, S8_PAD_BF16, S1_BF16, ONE_FRAME_BF16, TOPK1_BF16,
-         FIXED_TILES_BF16]
+         TOPK1_S4_BF16, FIXED_TILES_BF16]
 
 
 def _cuda_inputs(cfg, seed=0):
@@ -92,9 +95,11 @@ def test_pi3_32_frames_parity():
     assert tot_checked > 0
 
 
-@pytest.mark.parametrize("k", [64, 16, 8])
+@pytest.mark.parametrize("k", [128, 64, 40, 16, 8])
 def test_pi3_32_frames_other_topk(k):
-    """The list lengths of the ablation (top-8/16/64): the register-list kernels for k = 8, 16, 64."""
+    """The list lengths of the ablation (top-8/16/64) and of test-time adaptation
+    (top-128): one register-list pass for k <= 32, passes of 32 that continue the
+    sorted selection above that (k = 40: a second pass of 8)."""
     cfg = CONFIGS["pi3_f32"].with_(topk=k)
     x = _cuda_inputs(cfg)
     res = run_gpu(cfg, x)
@@ -103,6 +108,45 @@ def test_pi3_32_frames_other_topk(k):
         c, _ = compare_head(cfg, x, res, h)
         checked += c
     assert checked > 0
+
+
+@pytest.mark.parametrize("k", [40, 100])
+def test_topk_exact_ties_across_passes(k):
+    """Every frame holds the same tokens, so each region's score repeats exactly in
+    every frame and the k-th place falls inside a group of exact ties (32 frames:
+    k = 40 takes all 32 copies of one region and 8 of the next, across the boundary
+    of the first 32-entry pass).  Equal scores go to the lower region index in the
+    oracle and, the on-chip scores of identical regions being bitwise equal, on the
+    GPU too: the sets must be identical wherever the tie group at the k-th place is
+    separated from the neighbouring score values by more than 1e-3."""
+    cfg = CONFIGS["pi3_f32"].with_(num_heads=2, topk=k)
+    x = make_inputs(cfg, seed=4)
+    for n in ("q_img", "k_img", "v_img"):
+        x[n] = x[n][:, :1].expand_as(x[n]).contiguous()
+    x = {kk: v.cuda() for kk, v in x.items()}
+    res = run_gpu(cfg, x)
+    cand = np.ones(cfg.num_regions, dtype=bool)
+    exact = 0
+    for h in range(cfg.num_heads):
+        qc = oracle.pool(to_f64_numpy(x["q_img"][h]), cfg.grid_h, cfg.grid_w, cfg.pool_s)
+        kc = oracle.pool(to_f64_numpy(x["k_img"][h]), cfg.grid_h, cfg.grid_w, cfg.pool_s)
+        # one frame's scores, repeated: the copies of a region tie exactly (a blocked
+        # matmul over all columns could order the sums differently per column)
+        rpf = cfg.regions_per_frame
+        assert np.array_equal(kc, np.tile(kc[:rpf], (cfg.num_frames, 1)))
+        sc = np.tile(qc @ kc[:rpf].T, (1, cfg.num_frames))
+        want, _ = oracle.topk_rows(sc, cand, k)
+        got = res["idx"][h].cpu().numpy().astype(np.int64)
+        for r in range(cfg.num_regions):
+            v = sc[r, want[r, -1]]
+            above = sc[r][sc[r] > v]
+            below = sc[r][sc[r] < v]
+            sep = min((above.min() - v) if above.size else np.inf, (v - below.max()) if below.size else np.inf)
+            if sep > 1e-3 * abs(v):
+                assert sorted(got[r].tolist()) == sorted(want[r].tolist()), f"head {h} row {r}"
+                exact += 1
+        compare_head(cfg, x, res, h, windows=np.arange(0, cfg.num_regions, 37))
+    assert exact > cfg.num_regions // 2
 
 
 def _sample_windows(cfg, n, seed):
