@@ -318,10 +318,12 @@ __device__ __forceinline__ void topk_insert(float (&ts)[KC > 0 ? KC : 1], int (&
   }
 }
 
-// EX (top-k beyond one list, passes after the first): columns at or ahead of the
-// previous pass's last selection (a.excl_s / a.excl_i) in the order (score desc,
-// index asc) are not candidates, so the pass continues the sorted selection.
-template <int KC, bool GO, bool EX = false>
+// MP (top-k beyond one 32-entry list): 0 a single pass; 1 the first of several
+// passes; 2 a later pass, in which columns at or ahead of the previous pass's last
+// selection (a.excl_s / a.excl_i) in the order (score desc, index asc) are not
+// candidates, so the pass continues the sorted selection.  Passes 1 and 2 write
+// their last selection (a.last_s / a.last_i) when asked.
+template <int KC, bool GO, int MP = 0>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qlo,
                    const __grid_constant__ CUtensorMap tm_k0, const __grid_constant__ CUtensorMap tm_v0,
@@ -491,9 +493,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       ti[p] = -1;
     }
     bool ok = true;
-    float ex_s = INFINITY;                            // EX: the previous pass's last selection
+    float ex_s = INFINITY;                            // MP 2: the previous pass's last selection
     int ex_i = -1;
-    if constexpr (EX) {
+    if constexpr (MP == 2) {
       if (row < a.n_q) {
         ex_s = a.excl_s[static_cast<long long>(h) * a.n_q + row];
         ex_i = a.excl_i[static_cast<long long>(h) * a.n_q + row];
@@ -595,7 +597,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 notmax[c] = (cb[c] & fb) != 0u;
                 cb[c] &= ~fb;
               }
-              if constexpr (EX) {
+              if constexpr (MP == 2) {
                 if (cmax >= ex_s) {
                   // an earlier pass took these: score above its last, or equal at a lower index
                   const int col0 = static_cast<int>(kb) + 64 * hf + 32 * c;
@@ -722,7 +724,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         *reinterpret_cast<float2*>(a.part_ml + pr * 2) = make_float2(m, l);
       }
       if constexpr (L::TOPK) {
-        const long long base = (static_cast<long long>(h) * a.n_q + row) * a.cand_stride + a.cand_off;
+        const long long base = MP == 0 ? (static_cast<long long>(h) * a.n_q + row) * a.kc
+                                       : (static_cast<long long>(h) * a.n_q + row) * a.cand_stride + a.cand_off;
 #pragma unroll
         for (int p = 0; p < KC; ++p) {
           if (p < a.kc) {
@@ -730,7 +733,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (a.cand_user) a.cand_user[base + p] = ti[p];
           }
         }
-        if (a.last_s) {
+        if (MP != 0 && a.last_s) {
           // the last selection of this pass, where the next pass continues
           a.last_s[static_cast<long long>(h) * a.n_q + row] = kth_score<KC>(ts, a.kc);
           int li = ti[KC - 1];
@@ -778,13 +781,13 @@ bool make_map(CUtensorMap* m, const void* base, long long rows) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int KC, bool GO, bool EX = false>
+template <int KC, bool GO, int MP = 0>
 cudaError_t launch_kc(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t st) {
   const int sm = Lay<KC, GO>::BYTES;
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<KC, GO, EX>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<KC, GO, MP>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
   if (e != cudaSuccess) return e;
   dim3 grid((a.n_q + 2 * TBM - 1) / (2 * TBM), a.n_split, a.H);
-  attn_tc_kernel<KC, GO, EX><<<grid, NTHREADS, sm, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], a);
+  attn_tc_kernel<KC, GO, MP><<<grid, NTHREADS, sm, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], a);
   return cudaGetLastError();
 }
 
@@ -1430,7 +1433,12 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
   maps[6] = maps[2];
   if (a.kc > 0 && !make_map(&maps[6], a.k_lo, H * a.n_k[0])) return cudaErrorInvalidValue;
   if (a.kc == 0) return launch_kc<0, false>(a, maps, st);
-  if (a.excl_s) return (a.guide_only && a.kc <= 32) ? launch_kc<32, true, true>(a, maps, st) : cudaErrorInvalidValue;
+  if (a.excl_s) return (a.guide_only && a.kc <= 32) ? launch_kc<32, true, 2>(a, maps, st) : cudaErrorInvalidValue;
+  if (a.last_s) {
+    // the first of several passes (32 regions)
+    if (a.kc != 32) return cudaErrorInvalidValue;
+    return a.guide_only ? launch_kc<32, true, 1>(a, maps, st) : launch_kc<32, false, 1>(a, maps, st);
+  }
   if (a.kc <= 8) return launch_kc2<8>(a, maps, st);
   if (a.kc <= 16) return launch_kc2<16>(a, maps, st);
   if (a.kc <= 32) return launch_kc2<32>(a, maps, st);

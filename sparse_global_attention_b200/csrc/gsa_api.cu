@@ -93,7 +93,7 @@ struct Layout {
   size_t kbits_dense_words;
   // bf16 selection on tensor cores (s = 4): window order of the groups (written
   // once at create), and per forward the union of each group's selected regions
-  size_t winof, uni, ucnt;
+  size_t winof, grpof, uni, ucnt;
   int ngroups;
 };
 
@@ -138,6 +138,7 @@ Layout make_layout(const gsa_config* c, const Derived& d) {
   L.kbits_dense = L.kbits_dense_words ? take(L.kbits_dense_words * 4) : SIZE_MAX;
   L.ngroups = sel_on_tc(c, d) ? sel_group_count(d.R) : 0;
   L.winof = L.ngroups ? take(static_cast<size_t>(d.R) * 4) : SIZE_MAX;
+  L.grpof = L.ngroups ? take(static_cast<size_t>(L.ngroups) * 4) : SIZE_MAX;
   L.uni = L.ngroups ? take(static_cast<size_t>(c->num_heads) * L.ngroups * SEL_GROUP * c->topk * 8) : SIZE_MAX;
   L.ucnt = L.ngroups ? take(static_cast<size_t>(c->num_heads) * L.ngroups * 4) : SIZE_MAX;
   L.total = off;
@@ -289,7 +290,10 @@ int gsa_create(const gsa_config* cfg, gsa_ctx** out) {
   if (c->L.ngroups) {
     std::vector<int> order(static_cast<size_t>(d.R));
     sel_group_order(cfg->num_frames, cfg->pad_h / cfg->pool_s, cfg->pad_w / cfg->pool_s, order.data());
-    if (cudaMemcpy(c->ws + c->L.winof, order.data(), order.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess) {
+    std::vector<int> sched(static_cast<size_t>(c->L.ngroups));
+    sel_group_schedule(cfg->num_frames, d.rpf, c->L.ngroups, sched.data());
+    if (cudaMemcpy(c->ws + c->L.winof, order.data(), order.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(c->ws + c->L.grpof, sched.data(), sched.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess) {
       cudaFree(c->ws);
       delete c;
       return GSA_ERR_CUDA;
@@ -595,6 +599,7 @@ int forward_heads(gsa_ctx* c, int h0, int nh, const void* q_spec, const void* k_
       ta.q_img = q_img; ta.k_img = k_img; ta.v_img = v_img; ta.w_g = w_g;
       ta.idx = idx;
       ta.win_of = c->at<const int>(c->L.winof);
+      ta.grp_of = c->at<const int>(c->L.grpof);
       ta.NG = c->L.ngroups;
       ta.topk = cf.topk;
       ta.emax = SEL_GROUP * cf.topk;

@@ -60,20 +60,21 @@ struct AttnArgs {
   float* part_ml;            // [n_split][H][n_q][2]  (running max in raw score units, sum)
   // streaming top-k of the raw scores (compressed branch only)
   int kc;                    // regions kept per row by this launch (<= 32)
-  int* cand;                 // [H][n_q][cand_stride] region indices, best first, this launch's
-  int* cand_user;            //   kc of them from column cand_off; cand_user: optional copy
-  int cand_stride, cand_off;
-  // top-k beyond one launch's list: the launch continues the selection after the
-  // previous launch's last entry per row (excl_s score, excl_i region; guide-only
-  // launches only), and writes its own last entry to last_s / last_i if set
-  const float* excl_s;
-  const int* excl_i;
-  float* last_s;
-  int* last_i;
+  int* cand;                 // [H][n_q][kc] region indices, best first (with several passes:
+  int* cand_user;            //   [H][n_q][cand_stride], this launch's from column cand_off);
+                             //   cand_user: optional copy
   int rpf;                   // regions per frame
   int n_fixed;
   int fixed[MAX_FIXED];      // frames excluded from the candidates
   int* err;                  // device error word
+  // top-k in several passes of at most 32: every pass writes its last entry per row
+  // to last_s / last_i; a pass after the first (guide only) continues the selection
+  // after the previous pass's last entry (excl_s score, excl_i region)
+  int cand_stride, cand_off;
+  const float* excl_s;
+  const int* excl_i;
+  float* last_s;
+  int* last_i;
 };
 // tcgen05/TMEM/TMA version: 2 x 128 query rows per CTA, 128-key tiles; the
 // top-k runs when a.kc > 0 (a.q_lo / a.k_lo required)
@@ -133,6 +134,7 @@ struct SelTcArgs {
   const void* w_g;           // [H][64][64] bf16 (gate_mode 0)
   const int* idx;            // [H][R][topk] selected regions
   const int* win_of;         // [R] window at each group position (sel_group_order)
+  const int* grp_of;         // [NG] groups in processing order (sel_group_schedule)
   uint2* uni;                // [H][NG][emax] union entries: x region, y = (token bits << 16) | window bits
   int* ucnt;                 // [H][NG] distinct regions per group
   int emax;                  // SEL_GROUP * topk
@@ -153,6 +155,10 @@ int sel_group_count(int R);
 // group positions -> windows: per frame, row pairs top to bottom, walking the
 // columns alternately left to right and back (win_of has F * rows * cols entries)
 void sel_group_order(int F, int rows, int cols, int* win_of);
+// processing order of a head's groups: by the groups' position inside their frame
+// first, frame second, so that the groups in flight at once sit at the same place in
+// many frames and select overlapping regions (their K/V stays in L2)
+void sel_group_schedule(int F, int rpf, int NG, int* grp_of);
 cudaError_t launch_sel_union(const SelTcArgs& a, cudaStream_t st);
 cudaError_t launch_sel_tc(const SelTcArgs& a, cudaStream_t st);
 
