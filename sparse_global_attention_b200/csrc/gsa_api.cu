@@ -818,11 +818,17 @@ int gsa_backward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void*
   const size_t rows = static_cast<size_t>(H) * d.R;
   const size_t img = static_cast<size_t>(H) * d.img_per_head;
   const size_t sp = static_cast<size_t>(H) * d.spec_per_head;
-  // scratch: dO'_comp fp32 + bf16, D of compressed and special rows, dQ/dK/dV_comp, da
-  size_t off[8], tot = 0;
-  const size_t sz[8] = {rows * D * 4, rows * D * 2, rows * 4, sp * 4, rows * D * 4, rows * D * 4, rows * D * 4,
-                        img * D * 4};
-  for (int i = 0; i < 8; ++i) {
+  // scratch: dO'_comp fp32 + bf16, D of compressed and special rows, dQ/dK/dV_comp, da;
+  // with the fixed context computed apart (bf16 forward with fixed frames) also dO_sel
+  // (bf16), the union log-sum-exp and D of every image token, and dK/dV of the packed
+  // fixed keys
+  const long long nfix = c->L.nfix;
+  const size_t fk = static_cast<size_t>(H) * static_cast<size_t>(nfix);
+  size_t off[13], tot = 0;
+  const size_t sz[13] = {rows * D * 4, rows * D * 2, rows * 4, sp * 4, rows * D * 4, rows * D * 4, rows * D * 4,
+                         img * D * 4, nfix ? img * D * 2 : 0, nfix ? img * 4 : 0, nfix ? img * 4 : 0, fk * D * 4,
+                         fk * D * 4};
+  for (int i = 0; i < 13; ++i) {
     off[i] = tot;
     tot = align_up(tot + sz[i]);
   }
@@ -869,8 +875,40 @@ int gsa_backward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void*
   sb.gate_mode = gate; sb.dq = dq_img; sb.dk = dk_img; sb.dv = dv_img;
   sb.dk_spec = spec ? dk_spec : nullptr; sb.dv_spec = spec ? dv_spec : nullptr;
   sb.d_ocomp = docomp; sb.da = da;
+  if (nfix) {
+    // the forward attended the fixed context apart (its O_fix, LSE and packed K/V are
+    // still in the workspace): the selection backward takes the selected regions only
+    sa.fix_o = c->at<float>(c->L.ofix);
+    sa.fix_lse = c->at<float>(c->L.lsefix);
+    sb.dosel = reinterpret_cast<__nv_bfloat16*>(c->bw + off[8]);
+    sb.lse_u = reinterpret_cast<float*>(c->bw + off[9]);
+    sb.Dq = reinterpret_cast<float*>(c->bw + off[10]);
+  }
   if (launch_sel_bwd(sb, st) != cudaSuccess) return GSA_ERR_CUDA;
   prof.mark("bwd_selection_gate");
+  if (nfix) {
+    // the fixed context: dense attention backward of every image query over the packed
+    // fixed keys, P normalised over the union (its LSE from the selection backward);
+    // dq adds to the selection's, dK/dV go back to the fixed frames' tokens
+    const long long nq = d.img_per_head;
+    float* dkfix = reinterpret_cast<float*>(c->bw + off[11]);
+    float* dvfix = reinterpret_cast<float*>(c->bw + off[12]);
+    BwdArgs bf;
+    memset(&bf, 0, sizeof(bf));
+    bf.q = reinterpret_cast<const __nv_bfloat16*>(q_img); bf.q_hs = nq * D; bf.n_q = static_cast<int>(nq);
+    bf.nseg = 1;
+    bf.k[0] = c->at<__nv_bfloat16>(c->L.kfix); bf.v[0] = c->at<__nv_bfloat16>(c->L.vfix);
+    bf.kv_hs[0] = nfix * D; bf.n_k[0] = static_cast<int>(nfix); bf.kmask[0] = MASK_NONE;
+    bf.dO = sb.dosel; bf.do_hs = nq * D; bf.lse2 = sb.lse_u; bf.Dv = sb.Dq;
+    bf.dq = dq_img; bf.dq_hs = nq * D; bf.dq_accum = 1;
+    bf.dk[0] = dkfix; bf.dv[0] = dvfix; bf.dkv_hs[0] = nfix * D; bf.dkv_accum = 0;
+    bf.H = H; bf.g = g; bf.scale_log2 = scale * LOG2E; bf.scale = scale;
+    if (launch_attn_bwd_dq_tc(bf, err, st) != cudaSuccess || launch_attn_bwd_dkv_tc(bf, err, st) != cudaSuccess)
+      return GSA_ERR_CUDA;
+    if (launch_fixed_scatter_add(sa, dkfix, dvfix, dk_img, dv_img, dk_spec, dv_spec, st) != cudaSuccess)
+      return GSA_ERR_CUDA;
+    prof.mark("bwd_fixed_attn");
+  }
 
   // 2. compressed attention (split guide scores, as in the forward)
   const long long rhs = static_cast<long long>(d.R) * D;

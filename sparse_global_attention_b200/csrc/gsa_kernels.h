@@ -248,8 +248,21 @@ struct SelBwdArgs {
   float* dv_spec;
   float* d_ocomp;            // fp32 [H][R][64]: written
   float* da;                 // fp32 [H][F][Hp][Wp][64]: gate pre-activation gradient (0 on pads)
+  // fixed context computed apart (s.fix_o / s.fix_lse set, bf16): the kernel loops
+  // only the selected regions, with P normalised over the union of both key sets,
+  // and writes per image token what the dense backward over the fixed keys needs:
+  // dO_sel (bf16, 0 on pads), the union's base-2 log-sum-exp (+inf on pads) and
+  // D = dO_sel . O_sel
+  __nv_bfloat16* dosel;      // [H][F*Hp*Wp][64]
+  float* lse_u;              // [H][F*Hp*Wp]
+  float* Dq;                 // [H][F*Hp*Wp]
 };
 cudaError_t launch_sel_bwd(const SelBwdArgs& a, cudaStream_t st);
+// gradients of the packed fixed-context keys/values ([H][n_fixed * (ns + Hv*Wv)][64]
+// fp32, the layout of launch_fixed_gather) added to the fixed frames' special and
+// image tokens
+cudaError_t launch_fixed_scatter_add(const SelArgs& a, const float* dkfix, const float* dvfix, float* dk_img,
+                                     float* dv_img, float* dk_spec, float* dv_spec, cudaStream_t st);
 
 // pool backward and small steps
 struct PoolBwdArgs {

@@ -501,8 +501,10 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
                : "memory");
 }
 
-template <int S>
-__global__ void __launch_bounds__(SB_WARPS * 32) sel_bwd_kernel(const SelBwdArgs b) {
+// FSPLIT: the forward attended the fixed context apart (s.fix_o set); this kernel then
+// loops only the selected regions and leaves the fixed keys to the dense backward
+template <int S, bool FSPLIT>
+__device__ __forceinline__ void sel_bwd_body(const SelBwdArgs& b) {
   const SelArgs& a = b.s;
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -550,7 +552,9 @@ __global__ void __launch_bounds__(SB_WARPS * 32) sel_bwd_kernel(const SelBwdArgs
   cp_async_commit();
   __syncwarp();
   const int nk_dyn = a.topk * S * S;
-  const int nkeys = nk_dyn + a.n_fixed * (a.g.ns + a.g.Hp * a.g.Wp);
+  // with the fixed context computed apart only the selected regions are looped here
+  constexpr bool fsplit = FSPLIT;
+  const int nkeys = nk_dyn + (fsplit ? 0 : a.n_fixed * (a.g.ns + a.g.Hp * a.g.Wp));
   const int nblk = (nkeys + SEL_BN - 1) / SEL_BN;
   auto issue = [&](int blk, int st) {               // one key per lane, rows copied by 8 lanes
     const uint32_t sK = sKV + st * 2 * SEL_TILE;
@@ -675,6 +679,30 @@ __global__ void __launch_bounds__(SB_WARPS * 32) sel_bwd_kernel(const SelBwdArgs
     inv[rr] = qv[rr] ? 1.f / l[rr] : 0.f;
     lse[rr] = qv[rr] ? m[rr] * sl2 + __log2f(l[rr]) : INFINITY;   // +inf: P = 0 on pad rows
   }
+  if constexpr (fsplit) {
+    // the union with the fixed context: lse over both key sets, and O_sel as the
+    // weighted sum of the selected regions' and the fixed context's normalised outputs
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      float wd = 0.f, wf = 0.f;
+      const float* fo = a.fix_o + (static_cast<long long>(h) * a.F * a.g.Hp * a.g.Wp + tok[rr]) * D;
+      if (qv[rr]) {
+        const float lf = a.fix_lse[static_cast<long long>(h) * a.F * a.g.Hp * a.g.Wp + tok[rr]];
+        const float mm = fmaxf(lf, lse[rr]);
+        const float lu = mm + __log2f(ex2(lf - mm) + ex2(lse[rr] - mm));
+        wd = ex2(lse[rr] - lu);
+        wf = ex2(lf - lu);
+        lse[rr] = lu;
+      }
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        const float2 of = qv[rr] ? __ldg(reinterpret_cast<const float2*>(fo + 8 * nt + 2 * t)) : make_float2(0.f, 0.f);
+        o[nt][2 * rr] = o[nt][2 * rr] * inv[rr] * wd + of.x * wf;
+        o[nt][2 * rr + 1] = o[nt][2 * rr + 1] * inv[rr] * wd + of.y * wf;
+      }
+      inv[rr] = qv[rr] ? 1.f : 0.f;                  // o now holds the normalised O_sel
+    }
+  }
   float gg[8][4];                                   // g = sigmoid(W_g q) (or the forced gate)
 #pragma unroll
   for (int nt = 0; nt < 8; ++nt) gg[nt][0] = gg[nt][1] = gg[nt][2] = gg[nt][3] = 0.f;
@@ -733,6 +761,25 @@ __global__ void __launch_bounds__(SB_WARPS * 32) sel_bwd_kernel(const SelBwdArgs
   for (int rr = 0; rr < 2; ++rr) {
     Dr[rr] += __shfl_xor_sync(0xffffffffu, Dr[rr], 1);
     Dr[rr] += __shfl_xor_sync(0xffffffffu, Dr[rr], 2);
+  }
+  if constexpr (fsplit) {
+    // what the dense backward over the fixed keys reads, for every token of the window
+    const long long hq = static_cast<long long>(h) * a.F * a.g.Hp * a.g.Wp;
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      const int row = g + 8 * rr;
+      if (row >= S * S) continue;
+      const int y = wi * S + row / S, x = wj * S + row % S;
+      const long long tk = (static_cast<long long>(f) * a.g.Hp + y) * a.g.Wp + x;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+        *reinterpret_cast<uint32_t*>(b.dosel + (hq + tk) * D + 8 * nt + 2 * t) =
+            qv[rr] ? pack_bf16(o[nt][2 * rr], o[nt][2 * rr + 1]) : 0u;
+      if (t == 0) {
+        b.lse_u[hq + tk] = qv[rr] ? lse[rr] : INFINITY;
+        b.Dq[hq + tk] = qv[rr] ? Dr[rr] : 0.f;
+      }
+    }
   }
   // dO'_comp[r] = sum over the window's valid tokens of g dO (the window is region r)
 #pragma unroll
@@ -912,13 +959,33 @@ __global__ void __launch_bounds__(SB_WARPS * 32) sel_bwd_kernel(const SelBwdArgs
 }
 
 template <int S>
-cudaError_t launch_sel_bwd_s(const SelBwdArgs& b, cudaStream_t st) {
+__global__ void __launch_bounds__(SB_WARPS * 32) sel_bwd_kernel(const SelBwdArgs b) {
+  sel_bwd_body<S, false>(b);
+}
+// the fixed-context split keeps more values live; two CTAs per SM still
+template <int S>
+__global__ void __launch_bounds__(SB_WARPS * 32, 2) sel_bwd_fix_kernel(const SelBwdArgs b) {
+  sel_bwd_body<S, true>(b);
+}
+
+template <int S, bool FSPLIT>
+cudaError_t launch_sel_bwd_sf(const SelBwdArgs& b, cudaStream_t st) {
   const int sm = SB_WARPS * SB_WARP;
-  cudaError_t e = cudaFuncSetAttribute(sel_bwd_kernel<S>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+  auto kern = FSPLIT ? sel_bwd_fix_kernel<S> : sel_bwd_kernel<S>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
   if (e != cudaSuccess) return e;
   const long long w = static_cast<long long>(b.s.H) * b.s.R;
-  sel_bwd_kernel<S><<<static_cast<unsigned>((w + SB_WARPS - 1) / SB_WARPS), SB_WARPS * 32, sm, st>>>(b);
+  kern<<<static_cast<unsigned>((w + SB_WARPS - 1) / SB_WARPS), SB_WARPS * 32, sm, st>>>(b);
   return cudaGetLastError();
+}
+
+template <int S>
+cudaError_t launch_sel_bwd_s(const SelBwdArgs& b, cudaStream_t st) {
+  if (b.s.fix_o) {
+    if (!b.dosel || !b.lse_u || !b.Dq || !b.s.fix_lse) return cudaErrorInvalidValue;
+    return launch_sel_bwd_sf<S, true>(b, st);
+  }
+  return launch_sel_bwd_sf<S, false>(b, st);
 }
 
 }  // namespace
@@ -961,6 +1028,52 @@ __global__ void __launch_bounds__(256) fixed_gather_kernel(const SelArgs a, __nv
   reinterpret_cast<uint4*>(vfix + row * D)[c] = reinterpret_cast<const uint4*>(vs)[c];
 }
 }  // namespace
+
+namespace {
+// one thread per four channels of a fixed-context key row: its dK and dV added to the token
+__global__ void __launch_bounds__(256) fixed_scatter_kernel(const SelArgs a, const float* dkfix, const float* dvfix,
+                                                            float* dk_img, float* dv_img, float* dk_spec,
+                                                            float* dv_spec, int per_frame) {
+  const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long rows = static_cast<long long>(a.H) * a.n_fixed * per_frame;
+  if (gid >= rows * 16) return;
+  const int c = static_cast<int>(gid & 15);
+  const long long row = gid >> 4;
+  const int t = static_cast<int>(row % per_frame);
+  const long long hi = row / per_frame;
+  const int i = static_cast<int>(hi % a.n_fixed);
+  const int h = static_cast<int>(hi / a.n_fixed);
+  const int f = a.fixed[i];
+  float *kd, *vd;
+  if (t < a.g.ns) {
+    const long long o = ((static_cast<long long>(h) * a.F + f) * a.g.ns + t) * D;
+    kd = dk_spec + o;
+    vd = dv_spec + o;
+  } else {
+    const int u = t - a.g.ns, y = u / a.g.Wv, x = u - y * a.g.Wv;
+    const long long o = (((static_cast<long long>(h) * a.F + f) * a.g.Hp + y) * a.g.Wp + x) * D;
+    kd = dk_img + o;
+    vd = dv_img + o;
+  }
+  const float4 dk = reinterpret_cast<const float4*>(dkfix + row * D)[c];
+  const float4 dv = reinterpret_cast<const float4*>(dvfix + row * D)[c];
+  float4 k0 = reinterpret_cast<float4*>(kd)[c], v0 = reinterpret_cast<float4*>(vd)[c];
+  k0.x += dk.x; k0.y += dk.y; k0.z += dk.z; k0.w += dk.w;
+  v0.x += dv.x; v0.y += dv.y; v0.z += dv.z; v0.w += dv.w;
+  reinterpret_cast<float4*>(kd)[c] = k0;
+  reinterpret_cast<float4*>(vd)[c] = v0;
+}
+}  // namespace
+
+cudaError_t launch_fixed_scatter_add(const SelArgs& a, const float* dkfix, const float* dvfix, float* dk_img,
+                                     float* dv_img, float* dk_spec, float* dv_spec, cudaStream_t st) {
+  const int per_frame = a.g.ns + a.g.Hv * a.g.Wv;
+  const long long n = static_cast<long long>(a.H) * a.n_fixed * per_frame * 16;
+  if (n <= 0) return cudaSuccess;
+  fixed_scatter_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(a, dkfix, dvfix, dk_img, dv_img, dk_spec,
+                                                                               dv_spec, per_frame);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_fixed_gather(const SelArgs& a, __nv_bfloat16* kfix, __nv_bfloat16* vfix, cudaStream_t st) {
   const int per_frame = a.g.ns + a.g.Hv * a.g.Wv;

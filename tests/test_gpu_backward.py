@@ -23,7 +23,11 @@ VGGT = GSAConfig("bwd_pad_vggt", 5, 10, 11, 12, 12, 3, 2, 64, 4, 6, "bf16", (0, 
 # 600 regions and 528 special rows: five 128-row tiles each, so the three-stage
 # TMA rings of the tcgen05 dQ and dK/dV kernels wrap around
 WRAP = GSAConfig("bwd_ring_wrap", 24, 20, 20, 20, 20, 22, 2, 64, 4, 8, "bf16")
-CASES = [SMALL, MULTI, S2, VGGT, WRAP]
+# fixed context over seven 128-key tiles with a ragged last one (3 x (3 + 17*17) = 876
+# keys) on a padded grid with 2x2 windows: its dense backward (dQ added to the
+# selection's, dK/dV of the packed keys scattered back) over 1,944 query slots
+FIXED_TILES = GSAConfig("bwd_fixed_tiles", 6, 17, 17, 18, 18, 3, 2, 64, 2, 6, "bf16", (0, 2, 5))
+CASES = [SMALL, MULTI, S2, VGGT, WRAP, FIXED_TILES]
 
 
 def _close(name, got, want):
