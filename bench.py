@@ -576,6 +576,7 @@ def run_b200(args, cfg, rank, world, local, dist):
         ablations = {}
         specs = [("no_comp_value", dict(variant="no_comp_value")), ("no_selection", dict(variant="no_selection")),
                  ("top8", dict(topk=8)), ("top16", dict(topk=16)), ("top64", dict(topk=64)),
+                 ("top128", dict(topk=128)),
                  ("flashvggt_descriptor_attention", dict(variant="descriptor")), ("windows8x8", None)]
         for name, kw in specs:
             if kw is None:
@@ -651,7 +652,8 @@ def main():
                     help="also time gsa_backward (gradients of every input) on the same inputs")
     ap.add_argument("--ablations", action="store_true",
                     help="also time the layer variants of the ablation table (no compressed value, "
-                         "no selection, top-8/16/64) on the same inputs")
+                         "no selection, top-8/16/64, 8x8 windows), test-time top-128 and FlashVGGT's "
+                         "descriptor attention on the same inputs")
     ap.add_argument("--cpu-windows", type=int, default=2048)
     ap.add_argument("--ref-windows", type=int, default=512)
     args = ap.parse_args()
