@@ -654,8 +654,10 @@ def main():
                     help="also time the layer variants of the ablation table (no compressed value, "
                          "no selection, top-8/16/64, 8x8 windows), test-time top-128 and FlashVGGT's "
                          "descriptor attention on the same inputs")
-    ap.add_argument("--cpu-windows", type=int, default=2048)
-    ap.add_argument("--ref-windows", type=int, default=512)
+    # the same sample size for the cpu_baseline leg and the reference arm, so that
+    # their extrapolations agree
+    ap.add_argument("--cpu-windows", type=int, default=1024)
+    ap.add_argument("--ref-windows", type=int, default=1024)
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "b200":
         args.warmup = 3

@@ -58,6 +58,24 @@ def test_gate_modes_isolate_branches(cfg, mode):
         compare_head(cfg, x, res, h, gate_mode=mode)
 
 
+@pytest.mark.parametrize("cfg", [CONFIGS["tiny_fp32"], PAD_VGGT_BF16, S2_BF16],
+                         ids=["tiny_fp32", "pad_vggt_bf16", "s2_bf16"])
+def test_saturated_gate(cfg):
+    """W_g scaled up 40x: |W_g q| reaches tens, so g = sigmoid(W_g q) sits at 0 or 1
+    for most channels ([notes, 门控聚合]); the blend must follow the oracle's gate
+    there too (the tensor-core kernel forms g through tanh, the mma.sync kernel
+    through a clamped exp2)."""
+    x = make_inputs(cfg, seed=2)
+    x["w_g"] = (x["w_g"].float() * 40.0).to(x["w_g"].dtype)
+    q = to_f64_numpy(x["q_img"][0]).reshape(-1, 64)
+    gl = q @ to_f64_numpy(x["w_g"][0]).T
+    assert np.mean(np.abs(gl) > 10) > 0.4          # a large share of the channels saturated
+    x = {k: v.cuda() for k, v in x.items()}
+    res = run_gpu(cfg, x)
+    for h in range(cfg.num_heads):
+        compare_head(cfg, x, res, h)
+
+
 @pytest.mark.parametrize("cfg", [CONFIGS["tiny_fp32"], RAGGED_BF16, S2_BF16],
                          ids=["tiny_fp32", "ragged_bf16", "s2_bf16"])
 def test_selection_with_every_region_equals_dense(cfg):
