@@ -547,6 +547,17 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       float m = -INFINITY, l = 0.f;
       for (int t = 0; ok && t < nt; ++t) {
         const int Tt = T + t;
+        // the tile's eight regions, read while S is computed: bit e = one of the warp's
+        // windows chose region e, bit 8 + e = this row's window chose it, bit 16 = some
+        // region has tokens outside the valid grid
+        uint32_t tb = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int u = 8 * t + e;
+          const uint32_t y = u < nu ? ents[u].y : 0xffff0000u;
+          tb |= ((((y >> wsh) & 3u) != 0u ? 1u : 0u) << e) | (((y >> w) & 1u) << (8 + e)) |
+                ((y >> 16) != 0xffffu ? 0x10000u : 0u);
+        }
         ok = __all_sync(0xffffffffu, mbar_wait(bars.s_full(), Tt & 1, a.err));
         if (!ok) break;
         tc_fence_after();
@@ -555,37 +566,31 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         for (int hf = 0; hf < 2; ++hf) {
           uint32_t v[64];
           tmem_ld64(tS + 64 * hf, v);
-          // the half's four regions: window bits and token validity
-          uint32_t info[4];
-          uint32_t act = 0;                            // bit e: a region one of the warp's windows chose
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int u = 8 * t + 4 * hf + e;
-            info[e] = u < nu ? ents[u].y : 0u;
-            act |= (((info[e] >> wsh) & 3u) != 0u ? 1u : 0u) << e;
-          }
+          const uint32_t act = (tb >> (4 * hf)) & 15u, rsel = (tb >> (8 + 4 * hf)) & 15u;
           tmem_wait_ld();
           if (hf == 1) {
             tc_fence_before();
             warp_arrive(bars.s_free());
           }
           // a row takes a region only if its own window chose it: that enters the max
-          // as one select per region and the exponentials as an infinite offset; the
-          // regions with pad tokens (warp-uniform) mask those tokens one by one
-          float hmx = -INFINITY;
-          uint32_t rsel = 0;                           // bit e: this row's window chose region e
+          // as one select per region and the exponentials as an infinite offset; tiles
+          // with pad tokens (warp-uniform) mask those tokens one by one
+          if (tb & 0x10000u) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            if (act & (1u << e)) {
-              const uint32_t kv = info[e] >> 16;
+            for (int e = 0; e < 4; ++e) {
+              const int u = 8 * t + 4 * hf + e;
+              const uint32_t kv = u < nu ? ents[u].y >> 16 : 0xffffu;
               if (kv != 0xffffu) {
 #pragma unroll
                 for (int c = 0; c < 16; ++c) v[16 * e + c] = ((kv >> c) & 1u) ? v[16 * e + c] : 0xff800000u;
               }
-              const bool rs = ((info[e] >> w) & 1u) != 0u;
-              rsel |= (rs ? 1u : 0u) << e;
-              hmx = fmaxf(hmx, rs ? max16(v + 16 * e) : -INFINITY);
             }
+          }
+          float hmx = -INFINITY;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float mx = max16(v + 16 * e);
+            hmx = ((rsel >> e) & 1u) ? fmaxf(hmx, mx) : hmx;
           }
           // online softmax: the reference max moves only when this half raises the
           // row's max by more than 2^8
