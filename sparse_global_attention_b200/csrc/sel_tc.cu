@@ -548,15 +548,15 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       for (int t = 0; ok && t < nt; ++t) {
         const int Tt = T + t;
         // the tile's eight regions, read while S is computed: bit e = one of the warp's
-        // windows chose region e, bit 8 + e = this row's window chose it, bit 16 = some
-        // region has tokens outside the valid grid
+        // windows chose region e, bit 8 + e = this row's window chose it, bit 16 + e =
+        // region e has tokens outside the valid grid
         uint32_t tb = 0;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int u = 8 * t + e;
           const uint32_t y = u < nu ? ents[u].y : 0xffff0000u;
           tb |= ((((y >> wsh) & 3u) != 0u ? 1u : 0u) << e) | (((y >> w) & 1u) << (8 + e)) |
-                ((y >> 16) != 0xffffu ? 0x10000u : 0u);
+                ((y >> 16) != 0xffffu ? 1u << (16 + e) : 0u);
         }
         ok = __all_sync(0xffffffffu, mbar_wait(bars.s_full(), Tt & 1, a.err));
         if (!ok) break;
@@ -573,14 +573,14 @@ __global__ void __launch_bounds__(NTHREADS, 2)
             warp_arrive(bars.s_free());
           }
           // a row takes a region only if its own window chose it: that enters the max
-          // as one select per region and the exponentials as an infinite offset; tiles
-          // with pad tokens (warp-uniform) mask those tokens one by one
-          if (tb & 0x10000u) {
+          // as one select per region and the exponentials as an infinite offset; chosen
+          // regions with pad tokens (warp-uniform) mask those tokens one by one
+          const uint32_t pm = (tb >> (16 + 4 * hf)) & act;
+          if (pm) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int u = 8 * t + 4 * hf + e;
-              const uint32_t kv = u < nu ? ents[u].y >> 16 : 0xffffu;
-              if (kv != 0xffffu) {
+              if (pm & (1u << e)) {
+                const uint32_t kv = ents[8 * t + 4 * hf + e].y >> 16;
 #pragma unroll
                 for (int c = 0; c < 16; ++c) v[16 * e + c] = ((kv >> c) & 1u) ? v[16 * e + c] : 0xff800000u;
               }
@@ -637,11 +637,6 @@ __global__ void __launch_bounds__(NTHREADS, 2)
               }
             }
           }
-          // P is free once the previous tile's P V (of this or the previous group) has completed
-          if (hf == 0 && Tt > 0) {
-            ok = __all_sync(0xffffffffu, mbar_wait(bars.pv_done(), (Tt - 1) & 1, a.err));
-            if (!ok) break;
-          }
           const float mb = (m == -INFINITY) ? 0.f : m * sl2;
           uint32_t pk[32];
 #pragma unroll
@@ -658,6 +653,12 @@ __global__ void __launch_bounds__(NTHREADS, 2)
 #pragma unroll
               for (int c = 0; c < 8; ++c) pk[8 * e + c] = 0u;
             }
+          }
+          // P is free once the previous tile's P V (of this or the previous group) has
+          // completed: waited for only now, so that P V overlaps the exponentials
+          if (hf == 0 && Tt > 0) {
+            ok = __all_sync(0xffffffffu, mbar_wait(bars.pv_done(), (Tt - 1) & 1, a.err));
+            if (!ok) break;
           }
           tmem_st32(tP + 32 * hf, pk);
         }
