@@ -13,7 +13,7 @@
 // tile.  The group attends to the union of its windows' regions (about 83 of
 // the 256 selections are distinct at top-32, 2.6x the per-window work),
 // masked per window:
-//   sel_union_kernel  sorts the group's (region, window) pairs and writes each
+//   sel_union_kernel  one warp per group: sorts the group's (region, window) pairs and writes each
 //                     distinct region once with the bit set of windows that
 //                     chose it and the validity bits of its 16 tokens (pads);
 //   sel_tc_kernel     persistent, two CTAs per SM, each looping over groups.
@@ -183,17 +183,23 @@ __device__ __forceinline__ float sigmoid_tanh(float x) {
 // ---------------------------------------------------------------------------
 // union of a group's selections
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) sel_union_kernel(const SelTcArgs a) {
-  __shared__ uint32_t key[SEL_UNION_MAX];
-  __shared__ int wsum[8];
-  const int grp = blockIdx.x, h = blockIdx.y;
+// One warp per group, eight groups per CTA: the group's pairs sorted in the
+// warp's own shared-memory row, so every step synchronises a warp, not the CTA.
+constexpr int UNION_WARPS = 8;
+
+__global__ void __launch_bounds__(32 * UNION_WARPS) sel_union_kernel(const SelTcArgs a) {
+  __shared__ uint32_t keys[UNION_WARPS][SEL_UNION_MAX];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int grp = blockIdx.x * UNION_WARPS + warp, h = blockIdx.y;
+  if (grp >= a.NG) return;                         // no CTA-wide barrier follows
+  uint32_t* key = keys[warp];
   const int p0 = grp * GW;
   const int nw = min(GW, a.R - p0);
   const int k = a.topk;
   const int n = nw * k;
-  int np2 = 1;
+  int np2 = 2;
   while (np2 < n) np2 <<= 1;
-  for (int e = threadIdx.x; e < np2; e += blockDim.x) {
+  for (int e = lane; e < np2; e += 32) {
     uint32_t v = 0xffffffffu;
     if (e < n) {
       const int w = e / k, j = e - w * k;
@@ -206,11 +212,11 @@ __global__ void __launch_bounds__(256) sel_union_kernel(const SelTcArgs a) {
     }
     key[e] = v;
   }
-  __syncthreads();
+  __syncwarp();
   // bitonic sort, ascending: (region, window) pairs of one region end up adjacent
   for (int size = 2; size <= np2; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = threadIdx.x; i < (np2 >> 1); i += blockDim.x) {
+      for (int i = lane; i < (np2 >> 1); i += 32) {
         const int lo = 2 * i - (i & (stride - 1));
         const int hi = lo + stride;
         const bool up = (lo & size) == 0;
@@ -220,29 +226,25 @@ __global__ void __launch_bounds__(256) sel_union_kernel(const SelTcArgs a) {
           key[hi] = x;
         }
       }
-      __syncthreads();
+      __syncwarp();
     }
   }
-  // each thread takes a contiguous run of positions; the first pair of every
+  // each lane takes a contiguous run of positions; the first pair of every
   // region becomes one union entry
-  const int per = (np2 + blockDim.x - 1) / blockDim.x;
-  const int e0 = threadIdx.x * per, e1 = min(e0 + per, np2);
+  const int per = (np2 + 31) / 32;
+  const int e0 = min(lane * per, np2), e1 = min(e0 + per, np2);
   auto first = [&](int e) {
     return key[e] != 0xffffffffu && (e == 0 || (key[e] >> 3) != (key[e - 1] >> 3));
   };
   int cnt = 0;
   for (int e = e0; e < e1; ++e) cnt += first(e) ? 1 : 0;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int incl = cnt;
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
     const int y = __shfl_up_sync(0xffffffffu, incl, d);
     if (lane >= d) incl += y;
   }
-  if (lane == 31) wsum[warp] = incl;
-  __syncthreads();
   int off = incl - cnt;
-  for (int q = 0; q < warp; ++q) off += wsum[q];
   uint2* out = a.uni + (static_cast<long long>(h) * a.NG + grp) * a.emax;
   for (int e = e0; e < e1; ++e) {
     if (!first(e)) continue;
@@ -256,8 +258,8 @@ __global__ void __launch_bounds__(256) sel_union_kernel(const SelTcArgs a) {
     for (int dy = 0; dy < ly; ++dy) kv |= ((1u << lx) - 1u) << (4 * dy);
     out[off++] = make_uint2(reg, (kv << 16) | wm);
   }
-  // the last thread's end position is the number of distinct regions
-  if (threadIdx.x == blockDim.x - 1) a.ucnt[static_cast<long long>(h) * a.NG + grp] = off;
+  // the last lane's end position is the number of distinct regions
+  if (lane == 31) a.ucnt[static_cast<long long>(h) * a.NG + grp] = off;
 }
 
 // ---------------------------------------------------------------------------
@@ -826,8 +828,8 @@ void sel_group_schedule(int F, int rpf, int NG, int* grp_of) {
 
 cudaError_t launch_sel_union(const SelTcArgs& a, cudaStream_t st) {
   if (a.emax > SEL_UNION_MAX || a.topk * SEL_GROUP > a.emax) return cudaErrorInvalidValue;
-  dim3 grid(a.NG, a.H);
-  sel_union_kernel<<<grid, 256, 0, st>>>(a);
+  dim3 grid((a.NG + UNION_WARPS - 1) / UNION_WARPS, a.H);
+  sel_union_kernel<<<grid, 32 * UNION_WARPS, 0, st>>>(a);
   return cudaGetLastError();
 }
 
