@@ -152,7 +152,7 @@ GSA_API int gsa_forward(gsa_ctx *ctx,
  * dq/dk/dv_img [H][F][pad_h][pad_w][64] (0 on pads), dq/dk/dv_spec
  * [H][F][num_special][64] (unused when num_special = 0), dw_g [H][64][64]
  * (0 when the gate is forced).  bf16 contexts of the full layer with
- * pool_s <= 4 and topk <= 64 only (GSA_ERR_UNSUPPORTED otherwise); allocates a scratch of
+ * topk <= 64 only (GSA_ERR_UNSUPPORTED otherwise; every pool_s); allocates a scratch of
  * about 5 x H x R x 256 bytes plus one float per image-token channel on first
  * use (GSA_ERR_OOM if that fails), freed by gsa_destroy.  Asynchronous on
  * `stream`. */

@@ -807,7 +807,7 @@ int gsa_backward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void*
   const bool spec = cf.num_special > 0;
   if (spec && (!q_spec || !k_spec || !v_spec || !o_spec || !d_o_spec || !dq_spec || !dk_spec || !dv_spec))
     return GSA_ERR_INVALID_ARG;
-  if (d.fp32 || cf.variant != GSA_VARIANT_FULL || cf.pool_s > 4 || cf.topk > 64) return GSA_ERR_UNSUPPORTED;
+  if (d.fp32 || cf.variant != GSA_VARIANT_FULL || cf.topk > 64) return GSA_ERR_UNSUPPORTED;
   const int gate = effective_gate(cf);
   if (gate == GSA_GATE_LEARNED && !w_g) return GSA_ERR_INVALID_ARG;
   if (cf.num_fixed_frames > 0 && !spec) return GSA_ERR_INVALID_ARG;
@@ -857,6 +857,8 @@ int gsa_backward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void*
   // gradients reached by atomics or accumulation start at zero
   if (cudaMemsetAsync(dk_img, 0, img * D * 4, st) != cudaSuccess || cudaMemsetAsync(dv_img, 0, img * D * 4, st) != cudaSuccess)
     return GSA_ERR_CUDA;
+  // 8 x 8 windows span four warps of the selection backward, which add into dO'_comp
+  if (cf.pool_s == 8 && cudaMemsetAsync(docomp, 0, rows * D * 4, st) != cudaSuccess) return GSA_ERR_CUDA;
   if (spec && (cudaMemsetAsync(dk_spec, 0, sp * D * 4, st) != cudaSuccess ||
                cudaMemsetAsync(dv_spec, 0, sp * D * 4, st) != cudaSuccess))
     return GSA_ERR_CUDA;

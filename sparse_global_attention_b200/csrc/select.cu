@@ -518,8 +518,12 @@ __device__ __forceinline__ void sel_bwd_body(const SelBwdArgs& b) {
   int2* sReg = reinterpret_cast<int2*>(wbase + SB_REG);
   uint8_t* sValid = wbase + SB_VAL;
 
-  const long long win = static_cast<long long>(blockIdx.x) * SB_WARPS + warp;
-  if (win >= static_cast<long long>(a.H) * a.R) return;      // warp-uniform
+  // a window of s*s queries is RB blocks of 16 rows, one warp each (s = 8: four)
+  constexpr int RB = (S * S + 15) / 16;
+  const long long wrb = static_cast<long long>(blockIdx.x) * SB_WARPS + warp;
+  if (wrb >= static_cast<long long>(a.H) * a.R * RB) return;   // warp-uniform
+  const long long win = wrb / RB;
+  const int q0 = 16 * static_cast<int>(wrb - win * RB);       // the warp's first query of the window
   const int h = static_cast<int>(win / a.R);
   const int r = static_cast<int>(win - static_cast<long long>(h) * a.R);
   const long long img_hs = static_cast<long long>(a.F) * a.g.Hp * a.g.Wp * D;
@@ -543,11 +547,11 @@ __device__ __forceinline__ void sel_bwd_body(const SelBwdArgs& b) {
 #pragma unroll
   for (int it = 0; it < 4; ++it) {
     const int e = lane + 32 * it;
-    const int row = e >> 3, c = e & 7;
+    const int lrow = e >> 3, c = e & 7, row = q0 + lrow;
     const int y = wi * S + row / S, x = wj * S + row % S;
     const bool ok = row < S * S && y < a.g.Hv && x < a.g.Wv;
     const long long tok = ok ? (static_cast<long long>(f) * a.g.Hp + y) * a.g.Wp + x : 0;
-    cp_async16(sQ + swz(row, c), qh + tok * D + c * 8, ok ? 16 : 0);
+    cp_async16(sQ + swz(lrow, c), qh + tok * D + c * 8, ok ? 16 : 0);
   }
   cp_async_commit();
   __syncwarp();
@@ -672,7 +676,7 @@ __device__ __forceinline__ void sel_bwd_body(const SelBwdArgs& b) {
   for (int rr = 0; rr < 2; ++rr) {
     l[rr] += __shfl_xor_sync(0xffffffffu, l[rr], 1);
     l[rr] += __shfl_xor_sync(0xffffffffu, l[rr], 2);
-    const int row = g + 8 * rr;
+    const int row = q0 + g + 8 * rr;
     const int y = wi * S + row / S, x = wj * S + row % S;
     qv[rr] = row < S * S && y < a.g.Hv && x < a.g.Wv && l[rr] > 0.f;
     tok[rr] = (static_cast<long long>(f) * a.g.Hp + y) * a.g.Wp + x;
@@ -752,7 +756,7 @@ __device__ __forceinline__ void sel_bwd_body(const SelBwdArgs& b) {
       o[nt][2 * rr + 1] = dos1;
       gg[nt][2 * rr] = da0;                          // gg now holds da
       gg[nt][2 * rr + 1] = da1;
-      const int row = g + 8 * rr;
+      const int row = q0 + g + 8 * rr;
       if (row < S * S)
         *reinterpret_cast<float2*>(dah + tok[rr] * D + 8 * nt + 2 * t) = make_float2(da0, da1);
     }
@@ -767,7 +771,7 @@ __device__ __forceinline__ void sel_bwd_body(const SelBwdArgs& b) {
     const long long hq = static_cast<long long>(h) * a.F * a.g.Hp * a.g.Wp;
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
-      const int row = g + 8 * rr;
+      const int row = q0 + g + 8 * rr;
       if (row >= S * S) continue;
       const int y = wi * S + row / S, x = wj * S + row % S;
       const long long tk = (static_cast<long long>(f) * a.g.Hp + y) * a.g.Wp + x;
@@ -781,7 +785,8 @@ __device__ __forceinline__ void sel_bwd_body(const SelBwdArgs& b) {
       }
     }
   }
-  // dO'_comp[r] = sum over the window's valid tokens of g dO (the window is region r)
+  // dO'_comp[r] = sum over the window's valid tokens of g dO (the window is region r);
+  // a window of several row blocks adds its blocks' sums into a zeroed buffer
 #pragma unroll
   for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
@@ -795,8 +800,14 @@ __device__ __forceinline__ void sel_bwd_body(const SelBwdArgs& b) {
   if (g == 0) {
     float* dst = b.d_ocomp + (static_cast<long long>(h) * a.R + r) * D;
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-      *reinterpret_cast<float2*>(dst + 8 * nt + 2 * t) = make_float2(docs[nt][0], docs[nt][1]);
+    for (int nt = 0; nt < 8; ++nt) {
+      if constexpr (RB == 1) {
+        *reinterpret_cast<float2*>(dst + 8 * nt + 2 * t) = make_float2(docs[nt][0], docs[nt][1]);
+      } else {
+        atomicAdd(dst + 8 * nt + 2 * t, docs[nt][0]);
+        atomicAdd(dst + 8 * nt + 2 * t + 1, docs[nt][1]);
+      }
+    }
   }
   // dq from the gate: dq[k] = sum_c da[c] W_g[c][k] (B fragments from W_g's columns)
 #pragma unroll
@@ -946,7 +957,7 @@ __device__ __forceinline__ void sel_bwd_body(const SelBwdArgs& b) {
   float* dqh = b.dq + h * img_hs;
 #pragma unroll
   for (int rr = 0; rr < 2; ++rr) {
-    const int row = g + 8 * rr;
+    const int row = q0 + g + 8 * rr;
     if (row >= S * S) continue;
     const int y = wi * S + row / S, x = wj * S + row % S;
     const bool valid = y < a.g.Hv && x < a.g.Wv;
@@ -974,7 +985,7 @@ cudaError_t launch_sel_bwd_sf(const SelBwdArgs& b, cudaStream_t st) {
   auto kern = FSPLIT ? sel_bwd_fix_kernel<S> : sel_bwd_kernel<S>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
   if (e != cudaSuccess) return e;
-  const long long w = static_cast<long long>(b.s.H) * b.s.R;
+  const long long w = static_cast<long long>(b.s.H) * b.s.R * ((S * S + 15) / 16);   // warps
   kern<<<static_cast<unsigned>((w + SB_WARPS - 1) / SB_WARPS), SB_WARPS * 32, sm, st>>>(b);
   return cudaGetLastError();
 }
@@ -995,6 +1006,7 @@ cudaError_t launch_sel_bwd(const SelBwdArgs& b, cudaStream_t st) {
     case 1: return launch_sel_bwd_s<1>(b, st);
     case 2: return launch_sel_bwd_s<2>(b, st);
     case 4: return launch_sel_bwd_s<4>(b, st);
+    case 8: return launch_sel_bwd_s<8>(b, st);
     default: return cudaErrorInvalidValue;
   }
 }

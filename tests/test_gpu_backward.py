@@ -27,7 +27,12 @@ WRAP = GSAConfig("bwd_ring_wrap", 24, 20, 20, 20, 20, 22, 2, 64, 4, 8, "bf16")
 # keys) on a padded grid with 2x2 windows: its dense backward (dQ added to the
 # selection's, dK/dV of the packed keys scattered back) over 1,944 query slots
 FIXED_TILES = GSAConfig("bwd_fixed_tiles", 6, 17, 17, 18, 18, 3, 2, 64, 2, 6, "bf16", (0, 2, 5))
-CASES = [SMALL, MULTI, S2, VGGT, WRAP, FIXED_TILES]
+# 8x8 windows (the ablation's window size): each window's 64 queries are four row
+# blocks of the selection backward that add into the window's dO'_comp; a ragged grid,
+# and with fixed frames the split fixed-context backward
+S8 = GSAConfig("bwd_s8", 3, 14, 15, 16, 16, 2, 2, 64, 8, 3, "bf16")
+S8_FIXED = GSAConfig("bwd_s8_fixed", 4, 13, 16, 16, 16, 2, 2, 64, 8, 4, "bf16", (0, 2))
+CASES = [SMALL, MULTI, S2, VGGT, WRAP, FIXED_TILES, S8, S8_FIXED]
 
 
 def _close(name, got, want):
