@@ -1020,7 +1020,8 @@ __global__ void __launch_bounds__(BW_NTHREADS, 1)
       const int km = a.kmask[seg];
       uint32_t vm[4] = {~0u, ~0u, ~0u, ~0u};
       if (km != MASK_NONE || kb + TBN > nk) {
-        const uint4 t4 = tile_valid(km, a.g, nk, kb);
+        const uint32_t* kbits = a.kbits[seg];
+        const uint4 t4 = kbits ? __ldg(reinterpret_cast<const uint4*>(kbits) + (kb >> 7)) : tile_valid(km, a.g, nk, kb);
         vm[0] = t4.x; vm[1] = t4.y; vm[2] = t4.z; vm[3] = t4.w;
       }
 #pragma unroll 1

@@ -955,6 +955,7 @@ int gsa_backward(gsa_ctx* c, const void* q_spec, const void* k_spec, const void*
     bs.kv_hs[0] = shs; bs.n_k[0] = static_cast<int>(d.spec_per_head); bs.kmask[0] = MASK_NONE;
     bs.k[1] = reinterpret_cast<const __nv_bfloat16*>(k_img); bs.v[1] = reinterpret_cast<const __nv_bfloat16*>(v_img);
     bs.kv_hs[1] = ihs; bs.n_k[1] = static_cast<int>(d.img_per_head); bs.kmask[1] = d.pads ? MASK_IMG : MASK_NONE;
+    if (d.pads && c->L.kbits_words) bs.kbits[1] = c->at<const uint32_t>(c->L.kbits);   // the forward's table
     bs.dO = reinterpret_cast<const __nv_bfloat16*>(d_o_spec); bs.do_hs = shs;
     bs.lse2 = c->at<float>(c->L.lse_s); bs.Dv = Ds;
     bs.dq = dq_spec; bs.dq_hs = shs; bs.dq_accum = 0;

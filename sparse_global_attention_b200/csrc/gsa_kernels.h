@@ -227,6 +227,7 @@ struct BwdArgs {
   int H;
   Grid g;
   float scale_log2, scale;
+  const uint32_t* kbits[2];  // optional per-segment key validity, 4 words per 128-key tile (as the forward's)
 };
 // dQ on tcgen05/TMEM/TMA: 128 query rows per CTA; heads packed (q_hs = n_q * 64,
 // kv_hs = n_k * 64); split scores (q_lo, k_lo) with one key segment only
