@@ -29,6 +29,8 @@ CASES = [
     dict(F=4, grid=(5, 5), pad=(6, 6), ns=1, d=8, s=2, k=2, fixed=(1,), gate="learned"),
     dict(F=2, grid=(4, 4), pad=(4, 4), ns=2, d=8, s=2, k=2, fixed=(), gate="sel_only"),
     dict(F=2, grid=(4, 4), pad=(4, 4), ns=0, d=8, s=4, k=1, fixed=(), gate="comp_only"),
+    # 8x8 windows on a padded grid with a fixed frame (the GPU backward's four-row-block case)
+    dict(F=3, grid=(7, 8), pad=(8, 8), ns=1, d=8, s=8, k=1, fixed=(1,), gate="learned"),
 ]
 
 
@@ -44,7 +46,7 @@ def test_torch_forward_equals_numpy_oracle(c):
     np.testing.assert_allclose(o_spec.numpy(), ref["o_spec"].reshape(o_spec.shape), rtol=0, atol=1e-12)
 
 
-@pytest.mark.parametrize("c", CASES[:3])
+@pytest.mark.parametrize("c", CASES[:3] + CASES[4:])
 def test_gradients_match_central_differences(c):
     a = _inputs(c["F"], c["grid"], c["pad"], c["ns"], c["d"], 2, c["fixed"])
     kw = dict(grid_h=c["grid"][0], grid_w=c["grid"][1], pool_s=c["s"], fixed_frames=c["fixed"], gate_mode=c["gate"])
